@@ -1,0 +1,182 @@
+/*
+ * mlra.h -- C ABI of the MLRA / MLA latent-KV decode-attention library (libmlra.so).
+ *
+ * One decode step of one attention layer, in absorbed form, as described for
+ * Multi-Head Low-Rank Attention ("Multi-Head Low-Rank Attention", ai.info AI
+ * summary): Main Findings, "decoding reduces to three absorbable steps" --
+ *   1. query-side weight absorption           -> mlra_absorb_q
+ *   2. MQA-style attention over the shared latent KV cache, one softmax per
+ *      latent branch (Methodology, second paragraph), split over the KV
+ *      length (flash-decoding) and merged by log-sum-exp
+ *                                              -> mlra_decode_attn + mlra_splitkv_combine
+ *   3. output up-projection of every branch, summed over branches and scaled
+ *      by the branch-count rescale (Key Contributions #2 and #3)
+ *                                              -> mlra_out_proj
+ * n_blocks = 1 is MLA (one latent head, one softmax), the comparison mode.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Pointers.  Every tensor pointer is a CUDA device pointer owned by the caller.
+ *   The library allocates and frees no memory; scratch lives in a caller-owned
+ *   workspace (mlra_workspace_size).  Tensors are dense, row-major, in the
+ *   index order given, with no padding.
+ * Streams.  Every call only enqueues work on `stream` (0 = legacy default
+ *   stream) and returns; no call synchronises except mlra_get_device_error.
+ * Errors.  Invalid arguments are detected on the host and returned as a status
+ *   before anything is launched.  Launch failures return MLRA_ERR_CUDA.
+ *   Problems only the device can see (an out-of-range page id, an mbarrier wait
+ *   that exceeded its bound) are recorded in an error word inside the
+ *   workspace; kernels never trap.  Nothing throws across this ABI.
+ * Dtypes.  `dtype` is the storage type of the KV cache, W_uk, W_uv and
+ *   q_nope / q_rope (MLRA_F32 or MLRA_BF16).  Absorbed queries, split
+ *   partials, latent outputs, lse and the final output are always fp32.
+ *   Arithmetic accumulates in fp32 throughout.
+ * Index convention of the up-projections.  W[b, h, i, j] maps latent channel i
+ *   of block b to head-dim channel j of head h:
+ *     k_nope[t, j] = sum_i c_b[t, i] * W_uk[b, h, i, j]   (same for W_uv).
+ * Cache row of one token.  D = n_blocks*d_cb + d_r elements:
+ *   [ c_0 (d_cb) | c_1 (d_cb) | ... | c_{nb-1} (d_cb) | k_rope (d_r) ].
+ *   With d_h = 128 and four blocks of 128 plus d_r = 64 this is 576 elements,
+ *   4.5 d_h per token (Key Contributions #2; Main Findings, first bullet).
+ * Logit of head h, branch b, token t (Key Contributions #2; shared RoPE key):
+ *   z = (q_abs[h, b, :] . c_b[t] + q_rope[h, :] . k_rope[t]) * softmax_scale
+ */
+#ifndef MLRA_H_
+#define MLRA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mlra_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  MLRA_OK = 0,
+  MLRA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent dims      */
+  MLRA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (shape / dtype)      */
+  MLRA_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned               */
+  MLRA_ERR_WORKSPACE = 4,    /* workspace too small or misaligned              */
+  MLRA_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed            */
+  MLRA_ERR_BAD_PAGE = 6,     /* device: page id outside [0, num_pages)         */
+  MLRA_ERR_TIMEOUT = 7,      /* device: a bounded wait expired                 */
+  MLRA_ERR_NO_DEVICE = 8     /* no usable sm_100 device                        */
+} mlra_status_t;
+
+typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype_t;
+
+/* Shapes and scales of one attention layer. */
+typedef struct {
+  int32_t n_blocks;      /* latent branches nb: 4 (MLRA-4), 2 (MLRA-2), 1 (MLA)          */
+  int32_t d_cb;          /* width of one latent block c_b                                */
+  int32_t d_r;           /* width of the shared RoPE key (d_h / 2 in the paper's models) */
+  int32_t n_heads;       /* query heads h                                                */
+  int32_t d_h;           /* per-head NoPE key width = value width                        */
+  int32_t page_size;     /* tokens per cache page when paged (must be 64); else ignored  */
+  mlra_dtype_t dtype;    /* storage dtype, see above                                     */
+  float softmax_scale;   /* multiplies the logit, e.g. 1/sqrt(d_h + d_r)                 */
+  float branch_scale;    /* rescale of the summed branch outputs, e.g. 1/sqrt(n_blocks)  */
+} mlra_config_t;
+
+/* Human-readable name of a status code (static string). */
+const char* mlra_status_string(mlra_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t mlra_version(void);
+
+/*
+ * Step 1: query absorption (Main Findings, "three absorbable steps", first step).
+ *   q_abs[s, h, b, i] = sum_j W_uk[b, h, i, j] * q_nope[s, h, j]
+ * so that q_abs . c_b[t] equals q_nope . k_nope[t] with the explicit key.
+ *   q_nope : [batch, n_heads, d_h]            dtype
+ *   w_uk   : [n_blocks, n_heads, d_cb, d_h]   dtype
+ *   q_abs  : [batch, n_heads, n_blocks, d_cb] fp32 (written)
+ * fp32 accumulation.  batch = 0 is a no-op.
+ */
+mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const void* w_uk,
+                            float* q_abs, int32_t batch, mlra_stream_t stream);
+
+/*
+ * Workspace bytes needed by mlra_decode_attn / mlra_splitkv_combine for up to
+ * `batch` sequences on the current CUDA device (depends on its SM count).
+ * Writes the size to *bytes.  The workspace must be 256-byte aligned.  It holds
+ * the split plan, the split partials (fp32) and the device error word.
+ */
+mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t batch, size_t* bytes);
+
+/*
+ * Step 2a: split-KV attention over the latent cache, one softmax per branch.
+ * For every sequence s the tokens t in [0, seqlens[s]) are cut into chunks
+ * (planned on the device from seqlens, balanced over the SMs); for every chunk,
+ * head h and branch b it computes, over that chunk's tokens,
+ *   o_part = sum_t softmax(z)_t * c_b[t]        (latent output, fp32)
+ *   lse_part = log sum_t exp(z_t)               (natural log)
+ * and stores both in the workspace for mlra_splitkv_combine.
+ *   q_abs      : [batch, n_heads, n_blocks, d_cb] fp32 (from mlra_absorb_q)
+ *   q_rope     : [batch, n_heads, d_r] dtype
+ *   kv_cache   : paged (page_table != NULL): [num_pages, page_size, D] dtype;
+ *                contiguous (page_table == NULL): [batch, max_len, D] dtype
+ *   num_pages  : paged: pages in kv_cache (page ids are checked against it);
+ *                contiguous: ignored
+ *   page_table : [batch, max_pages] int32 or NULL.  Entry p of row s holds the
+ *                page of tokens [64p, 64p+64) of sequence s; entries past the
+ *                sequence's last page are never read.
+ *   max_pages  : paged: row stride of page_table; contiguous: max_len, the row
+ *                stride of kv_cache in tokens
+ *   seqlens    : [batch] int32, 0 <= seqlens[s] <= max_pages*page_size (paged)
+ *                or <= max_len (contiguous); device memory
+ *   workspace  : >= mlra_workspace_size bytes, 256-byte aligned, caller-owned
+ * Cache rows at or beyond seqlens[s] never influence the result, whatever they
+ * hold (they are zero-filled on chip before use).  The device error word is
+ * reset at the start of every call.  Pointers must be 16-byte aligned.
+ */
+mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, const void* q_rope,
+                               const void* kv_cache, int64_t num_pages, const int32_t* page_table,
+                               int32_t max_pages, const int32_t* seqlens, int32_t batch,
+                               void* workspace, size_t workspace_bytes, mlra_stream_t stream);
+
+/*
+ * Step 2b: merge the split partials of every (sequence, head, branch):
+ *   lse = log sum_k exp(lse_k);   o_lat = sum_k exp(lse_k - lse) * o_k
+ *   workspace : the one passed to the preceding mlra_decode_attn (same stream)
+ *   o_latent  : [batch, n_heads, n_blocks, d_cb] fp32 (written)
+ *   lse       : [batch, n_heads, n_blocks] fp32 natural log (written; may be NULL)
+ * A sequence with seqlens = 0 gets o_latent = 0 and lse = -inf.
+ */
+mlra_status_t mlra_splitkv_combine(const mlra_config_t* cfg, const void* workspace,
+                                   size_t workspace_bytes, int32_t batch, float* o_latent,
+                                   float* lse, mlra_stream_t stream);
+
+/*
+ * Step 3: output up-projection, summed over branches and rescaled
+ * (Key Contributions #2: block outputs are summed; #3: branch-count rescale):
+ *   out[s, h, j] = branch_scale * sum_b sum_i o_latent[s, h, b, i] * W_uv[b, h, i, j]
+ *   o_latent : [batch, n_heads, n_blocks, d_cb] fp32
+ *   w_uv     : [n_blocks, n_heads, d_cb, d_h] dtype
+ *   out      : [batch, n_heads, d_h] fp32 (written)
+ */
+mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, const void* w_uv,
+                            float* out, int32_t batch, mlra_stream_t stream);
+
+/*
+ * Read (and then clear) the device error word of a workspace.  Synchronises
+ * `stream`.  *device_status receives MLRA_OK or the first device-side error
+ * (MLRA_ERR_BAD_PAGE, MLRA_ERR_TIMEOUT) recorded since the last decode call.
+ */
+mlra_status_t mlra_get_device_error(const void* workspace, size_t workspace_bytes,
+                                    int32_t* device_status, mlra_stream_t stream);
+
+/*
+ * Which decode kernel mlra_decode_attn would launch for cfg on the current
+ * device: 1 = tensor-core kernel (tcgen05 / TMEM / TMA), 2 = fp32 SIMT kernel,
+ * 0 = unsupported.  Host-only query, launches nothing.
+ */
+int32_t mlra_decode_kernel_kind(const mlra_config_t* cfg);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLRA_H_ */
