@@ -1,0 +1,274 @@
+"""Python binding of libmlra.so: MLRA / MLA latent-KV decode attention on B200.
+
+Argument marshalling only: every step of the decode path runs in the library's
+CUDA kernels (see ``include/mlra.h`` for the operations, layouts and error
+behaviour).  PyTorch supplies device memory and the current stream.  There is
+no fallback: if the shared library is missing this module raises on import of
+the library handle, and every call requires CUDA tensors.
+
+Steps of one decode call ("Multi-Head Low-Rank Attention", Main Findings:
+decoding reduces to three absorbable steps):
+``absorb_q`` -> ``decode_attn`` -> ``splitkv_combine`` -> ``out_proj``.
+``Decoder`` bundles the four with preallocated buffers.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmlra.so")
+
+F32 = 0
+BF16 = 1
+
+STATUS = {
+    0: "MLRA_OK", 1: "MLRA_ERR_INVALID_ARG", 2: "MLRA_ERR_UNSUPPORTED", 3: "MLRA_ERR_ALIGNMENT",
+    4: "MLRA_ERR_WORKSPACE", 5: "MLRA_ERR_CUDA", 6: "MLRA_ERR_BAD_PAGE", 7: "MLRA_ERR_TIMEOUT",
+    8: "MLRA_ERR_NO_DEVICE",
+}
+
+# Every symbol the C header declares (checked by the CPU tests).
+EXPORTS = [
+    "mlra_status_string", "mlra_version", "mlra_absorb_q", "mlra_workspace_size",
+    "mlra_decode_attn", "mlra_splitkv_combine", "mlra_out_proj", "mlra_get_device_error",
+    "mlra_decode_kernel_kind",
+]
+
+
+class MlraError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class Config(ctypes.Structure):
+    """mirror of mlra_config_t"""
+    _fields_ = [
+        ("n_blocks", ctypes.c_int32), ("d_cb", ctypes.c_int32), ("d_r", ctypes.c_int32),
+        ("n_heads", ctypes.c_int32), ("d_h", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+        ("branch_scale", ctypes.c_float),
+    ]
+
+    @property
+    def D(self) -> int:
+        return self.n_blocks * self.d_cb + self.d_r
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.dtype == BF16 else torch.float32
+
+
+def make_config(n_blocks: int, d_cb: int, d_r: int, n_heads: int, d_h: int,
+                dtype: torch.dtype = torch.bfloat16, softmax_scale: Optional[float] = None,
+                branch_scale: Optional[float] = None, page_size: int = 64) -> Config:
+    """Config with the paper's default scales: 1/sqrt(d_h + d_r) and 1/sqrt(n_blocks)."""
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_h + d_r)
+    if branch_scale is None:
+        branch_scale = 1.0 / math.sqrt(n_blocks)
+    dt = {torch.bfloat16: BF16, torch.float32: F32}[dtype]
+    return Config(n_blocks, d_cb, d_r, n_heads, d_h, page_size, dt, softmax_scale, branch_scale)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmlra.so from this package directory (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} not found: build it with "
+                          "`python -m decode_attention_rank_mlra_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    CP = ctypes.POINTER(Config)
+    sig = {
+        "mlra_status_string": (ctypes.c_char_p, [I32]),
+        "mlra_version": (I32, []),
+        "mlra_absorb_q": (I32, [CP, P, P, P, I32, P]),
+        "mlra_workspace_size": (I32, [CP, I32, ctypes.POINTER(SZ)]),
+        "mlra_decode_attn": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, SZ, P]),
+        "mlra_splitkv_combine": (I32, [CP, P, SZ, I32, P, P, P]),
+        "mlra_out_proj": (I32, [CP, P, P, P, I32, P]),
+        "mlra_get_device_error": (I32, [P, SZ, ctypes.POINTER(I32), P]),
+        "mlra_decode_kernel_kind": (I32, [CP]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().mlra_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: Optional[torch.dtype] = None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise MlraError(fn, status)
+
+
+def absorb_q(cfg: Config, q_nope: torch.Tensor, w_uk: torch.Tensor,
+             q_abs: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Step 1: q_abs[s,h,b,i] = sum_j W_uk[b,h,i,j] q_nope[s,h,j] (fp32 out)."""
+    _need(q_nope, "q_nope", cfg.torch_dtype)
+    _need(w_uk, "w_uk", cfg.torch_dtype)
+    B = q_nope.shape[0]
+    if q_abs is None:
+        q_abs = torch.empty((B, cfg.n_heads, cfg.n_blocks, cfg.d_cb), dtype=torch.float32,
+                            device=q_nope.device)
+    _need(q_abs, "q_abs", torch.float32)
+    _check("mlra_absorb_q", lib().mlra_absorb_q(ctypes.byref(cfg), _ptr(q_nope), _ptr(w_uk),
+                                                _ptr(q_abs), B, _stream(stream)))
+    return q_abs
+
+
+def workspace_size(cfg: Config, batch: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mlra_workspace_size", lib().mlra_workspace_size(ctypes.byref(cfg), batch,
+                                                            ctypes.byref(n)))
+    return int(n.value)
+
+
+def alloc_workspace(cfg: Config, batch: int, device=None) -> torch.Tensor:
+    """Caller-owned workspace (uint8, 256-byte aligned by the caching allocator)."""
+    n = workspace_size(cfg, batch)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
+    off = (-ws.data_ptr()) % 256
+    return ws[off: off + n]
+
+
+def decode_attn(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor, kv_cache: torch.Tensor,
+                page_table: Optional[torch.Tensor], seqlens: torch.Tensor, max_pages: int,
+                workspace: torch.Tensor, stream=None) -> None:
+    """Step 2a: split-KV attention into the workspace.
+
+    Paged: kv_cache [num_pages, 64, D], page_table [B, max_pages] int32.
+    Contiguous: page_table None, kv_cache [B, max_len, D], max_pages = max_len.
+    """
+    _need(q_abs, "q_abs", torch.float32)
+    _need(q_rope, "q_rope", cfg.torch_dtype)
+    _need(kv_cache, "kv_cache", cfg.torch_dtype)
+    _need(seqlens, "seqlens", torch.int32)
+    _need(workspace, "workspace", torch.uint8)
+    num_pages = 0
+    if page_table is not None:
+        _need(page_table, "page_table", torch.int32)
+        num_pages = kv_cache.shape[0]
+    B = seqlens.shape[0]
+    _check("mlra_decode_attn", lib().mlra_decode_attn(
+        ctypes.byref(cfg), _ptr(q_abs), _ptr(q_rope), _ptr(kv_cache), num_pages, _ptr(page_table),
+        int(max_pages), _ptr(seqlens), B, _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def splitkv_combine(cfg: Config, workspace: torch.Tensor, batch: int,
+                    o_latent: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    stream=None):
+    """Step 2b: merge split partials -> o_latent [B,h,nb,d_cb], lse [B,h,nb] (fp32)."""
+    dev = workspace.device
+    if o_latent is None:
+        o_latent = torch.empty((batch, cfg.n_heads, cfg.n_blocks, cfg.d_cb), dtype=torch.float32,
+                               device=dev)
+    if lse is None:
+        lse = torch.empty((batch, cfg.n_heads, cfg.n_blocks), dtype=torch.float32, device=dev)
+    _need(o_latent, "o_latent", torch.float32)
+    _need(lse, "lse", torch.float32)
+    _check("mlra_splitkv_combine", lib().mlra_splitkv_combine(
+        ctypes.byref(cfg), _ptr(workspace), workspace.numel(), batch, _ptr(o_latent), _ptr(lse),
+        _stream(stream)))
+    return o_latent, lse
+
+
+def out_proj(cfg: Config, o_latent: torch.Tensor, w_uv: torch.Tensor,
+             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Step 3: out[s,h,:] = branch_scale * sum_b W_uv[b,h]^T o_latent[s,h,b] (fp32)."""
+    _need(o_latent, "o_latent", torch.float32)
+    _need(w_uv, "w_uv", cfg.torch_dtype)
+    B = o_latent.shape[0]
+    if out is None:
+        out = torch.empty((B, cfg.n_heads, cfg.d_h), dtype=torch.float32, device=o_latent.device)
+    _need(out, "out", torch.float32)
+    _check("mlra_out_proj", lib().mlra_out_proj(ctypes.byref(cfg), _ptr(o_latent), _ptr(w_uv),
+                                                _ptr(out), B, _stream(stream)))
+    return out
+
+
+def get_device_error(workspace: torch.Tensor, stream=None) -> int:
+    """Device-side status recorded in the workspace (synchronises the stream)."""
+    v = ctypes.c_int32(0)
+    _check("mlra_get_device_error", lib().mlra_get_device_error(
+        _ptr(workspace), workspace.numel(), ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+def decode_kernel_kind(cfg: Config) -> str:
+    k = lib().mlra_decode_kernel_kind(ctypes.byref(cfg))
+    return {0: "unsupported", 1: "tcgen05", 2: "simt"}[k]
+
+
+@dataclass
+class Decoder:
+    """One layer's decode step with preallocated outputs and workspace.
+
+    ``run`` launches absorb -> decode_attn -> splitkv_combine -> out_proj on
+    the current stream and returns ``out`` [B, h, d_h] fp32.
+    """
+
+    cfg: Config
+    batch: int
+    device: torch.device
+
+    def __post_init__(self):
+        c, B, dev = self.cfg, self.batch, self.device
+        self.workspace = alloc_workspace(c, B, dev)
+        self.q_abs = torch.empty((B, c.n_heads, c.n_blocks, c.d_cb), dtype=torch.float32, device=dev)
+        self.o_latent = torch.empty((B, c.n_heads, c.n_blocks, c.d_cb), dtype=torch.float32,
+                                    device=dev)
+        self.lse = torch.empty((B, c.n_heads, c.n_blocks), dtype=torch.float32, device=dev)
+        self.out = torch.empty((B, c.n_heads, c.d_h), dtype=torch.float32, device=dev)
+
+    def run(self, q_nope, q_rope, w_uk, w_uv, kv_cache, page_table, seqlens, max_pages,
+            stream=None) -> torch.Tensor:
+        absorb_q(self.cfg, q_nope, w_uk, self.q_abs, stream)
+        decode_attn(self.cfg, self.q_abs, q_rope, kv_cache, page_table, seqlens, max_pages,
+                    self.workspace, stream)
+        splitkv_combine(self.cfg, self.workspace, self.batch, self.o_latent, self.lse, stream)
+        out_proj(self.cfg, self.o_latent, w_uv, self.out, stream)
+        return self.out
+
+
+__all__ = [
+    "Config", "make_config", "lib", "absorb_q", "workspace_size", "alloc_workspace",
+    "decode_attn", "splitkv_combine", "out_proj", "get_device_error", "decode_kernel_kind",
+    "Decoder", "MlraError", "EXPORTS", "F32", "BF16",
+]

@@ -1,0 +1,232 @@
+// Host side of the C ABI declared in include/mlra.h: argument validation,
+// workspace layout, kernel selection and launches.  No allocation, no host
+// synchronisation (except mlra_get_device_error).
+#include "mlra_internal.cuh"
+
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+using namespace mlra;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int num_sms_current(int* dev_out) {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  if (dev_out) *dev_out = dev;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+bool device_is_sm100(int dev) {
+  static int cache[kMaxDevices] = {0};  // 0 unknown, 1 yes, 2 no
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  if (cache[dev] == 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cache[dev] == 1;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+mlra_status_t check_cfg(const mlra_config_t* c) {
+  if (!c) return MLRA_ERR_INVALID_ARG;
+  if (c->n_blocks < 1 || c->d_cb < 1 || c->d_r < 0 || c->n_heads < 1 || c->d_h < 1)
+    return MLRA_ERR_INVALID_ARG;
+  if (c->dtype != MLRA_F32 && c->dtype != MLRA_BF16) return MLRA_ERR_INVALID_ARG;
+  if (!(c->softmax_scale == c->softmax_scale) || !(c->branch_scale == c->branch_scale))
+    return MLRA_ERR_INVALID_ARG;  // NaN
+  if (c->d_h > 128 || (c->d_h % 8) != 0 || (c->d_cb % 8) != 0) return MLRA_ERR_UNSUPPORTED;
+  return MLRA_OK;
+}
+
+// 1 = tensor core, 2 = SIMT, 0 = unsupported.  MLRA_DECODE_KERNEL=simt forces
+// the SIMT kernel (used by tests to cross-check the two paths).
+int choose_kernel(const mlra_config_t& c, int dev) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* e = getenv("MLRA_DECODE_KERNEL");
+    forced = (e && strcmp(e, "simt") == 0) ? 2 : 0;
+  }
+  if (forced == 2) return simt_supported(c) ? 2 : 0;
+  if (c.dtype == MLRA_BF16 && device_is_sm100(dev) && tc_supported(c)) return 1;
+  if (simt_supported(c)) return 2;
+  return 0;
+}
+
+struct Grid { int kind, n_groups, ctas_per_group; };
+
+mlra_status_t plan_grid(const mlra_config_t& c, Grid* g) {
+  int dev = 0;
+  const int sms = num_sms_current(&dev);
+  if (sms <= 0) return MLRA_ERR_NO_DEVICE;
+  g->kind = choose_kernel(c, dev);
+  if (g->kind == 1) tc_grid(c, sms, &g->n_groups, &g->ctas_per_group);
+  else if (g->kind == 2) simt_grid(c, sms, &g->n_groups, &g->ctas_per_group);
+  else return MLRA_ERR_UNSUPPORTED;
+  return MLRA_OK;
+}
+
+WsLayout layout_for(const mlra_config_t& c, int batch, const Grid& g) {
+  return ws_layout(batch, c.n_heads, c.n_blocks, c.d_cb, batch + g.ctas_per_group);
+}
+
+mlra_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mlra_status_string(mlra_status_t s) {
+  switch (s) {
+    case MLRA_OK: return "ok";
+    case MLRA_ERR_INVALID_ARG: return "invalid argument";
+    case MLRA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MLRA_ERR_ALIGNMENT: return "pointer under-aligned";
+    case MLRA_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case MLRA_ERR_CUDA: return "CUDA error";
+    case MLRA_ERR_BAD_PAGE: return "page id out of range (device)";
+    case MLRA_ERR_TIMEOUT: return "bounded wait expired (device)";
+    case MLRA_ERR_NO_DEVICE: return "no usable CUDA device";
+  }
+  return "unknown status";
+}
+
+int32_t mlra_version(void) { return 10000; }
+
+int32_t mlra_decode_kernel_kind(const mlra_config_t* cfg) {
+  if (check_cfg(cfg) != MLRA_OK) return 0;
+  Grid g;
+  if (plan_grid(*cfg, &g) != MLRA_OK) return 0;
+  return g.kind;
+}
+
+mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const void* w_uk,
+                            float* q_abs, int32_t batch, mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0) return MLRA_ERR_INVALID_ARG;
+  if (batch == 0) return MLRA_OK;
+  if (!q_nope || !w_uk || !q_abs) return MLRA_ERR_INVALID_ARG;
+  return from_cuda(launch_absorb(*cfg, q_nope, w_uk, q_abs, batch, (cudaStream_t)stream));
+}
+
+mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t batch, size_t* bytes) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0 || !bytes) return MLRA_ERR_INVALID_ARG;
+  Grid g;
+  st = plan_grid(*cfg, &g);
+  if (st != MLRA_OK) return st;
+  *bytes = layout_for(*cfg, batch, g).total;
+  return MLRA_OK;
+}
+
+mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, const void* q_rope,
+                               const void* kv_cache, int64_t num_pages,
+                               const int32_t* page_table, int32_t max_pages,
+                               const int32_t* seqlens, int32_t batch, void* workspace,
+                               size_t workspace_bytes, mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0) return MLRA_ERR_INVALID_ARG;
+  if (!workspace) return MLRA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLRA_ERR_WORKSPACE;
+  if (batch > 0 && (!q_abs || !q_rope || !kv_cache || !seqlens)) return MLRA_ERR_INVALID_ARG;
+  if (max_pages < 1) return MLRA_ERR_INVALID_ARG;
+  if (page_table) {
+    if (cfg->page_size != kPageSize) return MLRA_ERR_UNSUPPORTED;
+    if (num_pages < 1 || num_pages > (int64_t(1) << 31) / kPageSize) return MLRA_ERR_INVALID_ARG;
+  }
+  const uintptr_t elt = cfg->dtype == MLRA_BF16 ? 2 : 4;
+  if (!aligned(kv_cache, 16) || !aligned(q_abs, 4) || !aligned(q_rope, elt) ||
+      !aligned(seqlens, 4) || (page_table && !aligned(page_table, 4)))
+    return MLRA_ERR_ALIGNMENT;
+  Grid g;
+  st = plan_grid(*cfg, &g);
+  if (st != MLRA_OK) return st;
+  const WsLayout L = layout_for(*cfg, batch, g);
+  if (workspace_bytes < L.total) return MLRA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t cap64 = page_table ? int64_t(max_pages) * kPageSize : int64_t(max_pages);
+  if (cap64 > (int64_t(1) << 30)) return MLRA_ERR_INVALID_ARG;
+  const int cap = (int)cap64;
+  cudaError_t e = launch_plan(seqlens, batch, cap, g.ctas_per_group, workspace, L, s);
+  if (e != cudaSuccess) return MLRA_ERR_CUDA;
+  if (batch == 0) return MLRA_OK;
+  DecodeArgs a;
+  a.cfg = *cfg;
+  a.q_abs = q_abs;
+  a.q_rope = q_rope;
+  a.kv_cache = kv_cache;
+  a.num_pages = page_table ? num_pages : 0;
+  a.page_table = page_table;
+  a.max_pages = max_pages;
+  a.cap = cap;
+  a.seqlens = seqlens;
+  a.batch = batch;
+  a.ws = workspace;
+  a.L = L;
+  a.ctas_per_group = g.ctas_per_group;
+  a.n_groups = g.n_groups;
+  e = (g.kind == 1) ? launch_decode_tc(a, s) : launch_decode_simt(a, s);
+  return from_cuda(e);
+}
+
+mlra_status_t mlra_splitkv_combine(const mlra_config_t* cfg, const void* workspace,
+                                   size_t workspace_bytes, int32_t batch, float* o_latent,
+                                   float* lse, mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0 || !workspace) return MLRA_ERR_INVALID_ARG;
+  if (batch == 0) return MLRA_OK;
+  if (!o_latent) return MLRA_ERR_INVALID_ARG;
+  Grid g;
+  st = plan_grid(*cfg, &g);
+  if (st != MLRA_OK) return st;
+  const WsLayout L = layout_for(*cfg, batch, g);
+  if (workspace_bytes < L.total) return MLRA_ERR_WORKSPACE;
+  return from_cuda(launch_combine(*cfg, workspace, L, batch, o_latent, lse, (cudaStream_t)stream));
+}
+
+mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, const void* w_uv,
+                            float* out, int32_t batch, mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0) return MLRA_ERR_INVALID_ARG;
+  if (batch == 0) return MLRA_OK;
+  if (!o_latent || !w_uv || !out) return MLRA_ERR_INVALID_ARG;
+  return from_cuda(launch_out_proj(*cfg, o_latent, w_uv, out, batch, (cudaStream_t)stream));
+}
+
+mlra_status_t mlra_get_device_error(const void* workspace, size_t workspace_bytes,
+                                    int32_t* device_status, mlra_stream_t stream) {
+  if (!workspace || !device_status || workspace_bytes < sizeof(WsHeader))
+    return MLRA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return MLRA_ERR_CUDA;
+  *device_status = v;
+  if (v != 0) {
+    e = cudaMemsetAsync(const_cast<void*>(workspace), 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return MLRA_ERR_CUDA;
+  }
+  return MLRA_OK;
+}
+
+}  // extern "C"

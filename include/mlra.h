@@ -47,6 +47,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define MLRA_API __attribute__((visibility("default")))
+#else
+#define MLRA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -57,7 +63,7 @@ typedef enum {
   MLRA_OK = 0,
   MLRA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent dims      */
   MLRA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (shape / dtype)      */
-  MLRA_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned               */
+  MLRA_ERR_ALIGNMENT = 3,    /* a pointer is under-aligned (see each call)     */
   MLRA_ERR_WORKSPACE = 4,    /* workspace too small or misaligned              */
   MLRA_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed            */
   MLRA_ERR_BAD_PAGE = 6,     /* device: page id outside [0, num_pages)         */
@@ -81,10 +87,10 @@ typedef struct {
 } mlra_config_t;
 
 /* Human-readable name of a status code (static string). */
-const char* mlra_status_string(mlra_status_t status);
+MLRA_API const char* mlra_status_string(mlra_status_t status);
 
 /* Library version as major*10000 + minor*100 + patch. */
-int32_t mlra_version(void);
+MLRA_API int32_t mlra_version(void);
 
 /*
  * Step 1: query absorption (Main Findings, "three absorbable steps", first step).
@@ -95,7 +101,7 @@ int32_t mlra_version(void);
  *   q_abs  : [batch, n_heads, n_blocks, d_cb] fp32 (written)
  * fp32 accumulation.  batch = 0 is a no-op.
  */
-mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const void* w_uk,
+MLRA_API mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const void* w_uk,
                             float* q_abs, int32_t batch, mlra_stream_t stream);
 
 /*
@@ -104,7 +110,7 @@ mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const 
  * Writes the size to *bytes.  The workspace must be 256-byte aligned.  It holds
  * the split plan, the split partials (fp32) and the device error word.
  */
-mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t batch, size_t* bytes);
+MLRA_API mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t batch, size_t* bytes);
 
 /*
  * Step 2a: split-KV attention over the latent cache, one softmax per branch.
@@ -130,9 +136,11 @@ mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t batch, size_
  *   workspace  : >= mlra_workspace_size bytes, 256-byte aligned, caller-owned
  * Cache rows at or beyond seqlens[s] never influence the result, whatever they
  * hold (they are zero-filled on chip before use).  The device error word is
- * reset at the start of every call.  Pointers must be 16-byte aligned.
+ * reset at the start of every call.  kv_cache must be 16-byte aligned (it is
+ * read by the tensor-memory accelerator); the other pointers need only the
+ * alignment of their element type.
  */
-mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, const void* q_rope,
+MLRA_API mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, const void* q_rope,
                                const void* kv_cache, int64_t num_pages, const int32_t* page_table,
                                int32_t max_pages, const int32_t* seqlens, int32_t batch,
                                void* workspace, size_t workspace_bytes, mlra_stream_t stream);
@@ -145,7 +153,7 @@ mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, con
  *   lse       : [batch, n_heads, n_blocks] fp32 natural log (written; may be NULL)
  * A sequence with seqlens = 0 gets o_latent = 0 and lse = -inf.
  */
-mlra_status_t mlra_splitkv_combine(const mlra_config_t* cfg, const void* workspace,
+MLRA_API mlra_status_t mlra_splitkv_combine(const mlra_config_t* cfg, const void* workspace,
                                    size_t workspace_bytes, int32_t batch, float* o_latent,
                                    float* lse, mlra_stream_t stream);
 
@@ -157,7 +165,7 @@ mlra_status_t mlra_splitkv_combine(const mlra_config_t* cfg, const void* workspa
  *   w_uv     : [n_blocks, n_heads, d_cb, d_h] dtype
  *   out      : [batch, n_heads, d_h] fp32 (written)
  */
-mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, const void* w_uv,
+MLRA_API mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, const void* w_uv,
                             float* out, int32_t batch, mlra_stream_t stream);
 
 /*
@@ -165,7 +173,7 @@ mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, con
  * `stream`.  *device_status receives MLRA_OK or the first device-side error
  * (MLRA_ERR_BAD_PAGE, MLRA_ERR_TIMEOUT) recorded since the last decode call.
  */
-mlra_status_t mlra_get_device_error(const void* workspace, size_t workspace_bytes,
+MLRA_API mlra_status_t mlra_get_device_error(const void* workspace, size_t workspace_bytes,
                                     int32_t* device_status, mlra_stream_t stream);
 
 /*
@@ -173,7 +181,7 @@ mlra_status_t mlra_get_device_error(const void* workspace, size_t workspace_byte
  * device: 1 = tensor-core kernel (tcgen05 / TMEM / TMA), 2 = fp32 SIMT kernel,
  * 0 = unsupported.  Host-only query, launches nothing.
  */
-int32_t mlra_decode_kernel_kind(const mlra_config_t* cfg);
+MLRA_API int32_t mlra_decode_kernel_kind(const mlra_config_t* cfg);
 
 #ifdef __cplusplus
 }

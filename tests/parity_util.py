@@ -1,0 +1,78 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path, compare to the oracle."""
+from __future__ import annotations
+
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+import decode_attention_rank_mlra_b200 as mlra
+import oracle
+import workloads as W
+
+# Tolerances (stated by the task for this method):
+#   fp32 cache: normwise max relative error <= 1e-5;
+#   bf16 cache (fp32 accumulation, oracle on the same bf16-rounded inputs):
+#   max|err| <= 5e-3 * max|ref| and mean|err| <= 5e-4 * mean|ref|.
+F32_MAX_REL = 1e-5
+BF16_MAX = 5e-3
+BF16_MEAN = 5e-4
+
+
+def config_of(spec: W.WorkloadSpec) -> mlra.Config:
+    return mlra.make_config(spec.n_blocks, spec.d_cb, spec.d_r, spec.n_heads, spec.d_h,
+                            dtype=spec.torch_dtype, softmax_scale=spec.softmax_scale,
+                            branch_scale=spec.branch_scale)
+
+
+def run_gpu(inp: W.DecodeInputs) -> Dict[str, torch.Tensor]:
+    """Full decode step through the C ABI; returns CPU copies of every output."""
+    spec = inp.spec
+    cfg = config_of(spec)
+    dec = mlra.Decoder(cfg, spec.batch, inp.device)
+    max_pages = inp.page_table.shape[1] if inp.page_table is not None else inp.max_len
+    dec.run(inp.q_nope, inp.q_rope, inp.w_uk, inp.w_uv, inp.kv_cache, inp.page_table,
+            inp.seqlens, max_pages)
+    err = mlra.get_device_error(dec.workspace)
+    torch.cuda.synchronize()
+    return dict(out=dec.out.cpu(), o_lat=dec.o_latent.cpu(), lse=dec.lse.cpu(),
+                q_abs=dec.q_abs.cpu(), device_error=err)
+
+
+def check_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = "out"):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    if dtype == "f32":
+        rel = err.max() / max(np.abs(ref).max(), 1e-30)
+        assert rel <= F32_MAX_REL, f"{what}: max rel err {rel:.3e} > {F32_MAX_REL}"
+        return dict(max_rel=rel)
+    mx = err.max() / max(np.abs(ref).max(), 1e-30)
+    mn = err.mean() / max(np.abs(ref).mean(), 1e-30)
+    assert mx <= BF16_MAX, f"{what}: max err {mx:.3e} * max|ref| > {BF16_MAX}"
+    assert mn <= BF16_MEAN, f"{what}: mean err {mn:.3e} * mean|ref| > {BF16_MEAN}"
+    return dict(max_rel=mx, mean_rel=mn)
+
+
+def compare_batch(inp: W.DecodeInputs, got: Dict[str, torch.Tensor],
+                  seqs: Optional[Sequence[int]] = None, heads: Optional[Sequence[int]] = None):
+    """Oracle on (a subset of) the same inputs; compare out, o_lat, lse."""
+    spec = inp.spec
+    seqs = list(range(spec.batch)) if seqs is None else list(seqs)
+    hs = list(range(spec.n_heads)) if heads is None else list(heads)
+    refs = oracle.decode_batch(inp, heads=hs, seqs=seqs)
+    out_ref = np.stack([r.out[hs] for r in refs])
+    out_got = got["out"].double().numpy()[seqs][:, hs]
+    stats = check_close(out_got, out_ref, spec.dtype, "out")
+    lat_ref = np.stack([r.o_lat[hs] for r in refs])
+    lat_got = got["o_lat"].double().numpy()[seqs][:, hs]
+    check_close(lat_got, lat_ref, spec.dtype, "o_lat")
+    lse_ref = np.stack([r.lse[hs] for r in refs])
+    lse_got = got["lse"].double().numpy()[seqs][:, hs]
+    finite = np.isfinite(lse_ref)
+    assert np.array_equal(finite, np.isfinite(lse_got))
+    if finite.any():
+        assert np.max(np.abs(lse_got[finite] - lse_ref[finite])) < (1e-5 if spec.dtype == "f32" else 2e-3)
+    return stats

@@ -1,0 +1,176 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Oracle-sized cases span several 64-token tiles and a ragged tail; full-size
+workloads are checked on sampled (sequence, head) outputs regenerated alone.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_rank_mlra_b200 as mlra
+import oracle
+import workloads as W
+from parity_util import check_close, compare_batch, config_of, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from decode_attention_rank_mlra_b200 import build
+    build.build()
+    torch.cuda.init()
+
+
+def _small(name, batch, seqlens, heads=None, seed=11):
+    spec = W.WORKLOADS[name]
+    s = W.scaled_down(spec, batch, seqlen=int(max(seqlens)), n_heads=heads, seed=seed)
+    return W.make_inputs(s, "cuda", seqlens=np.asarray(seqlens, np.int32))
+
+
+def test_fp32_workload_full():
+    """B=1, h=4, d_h=64, L=256, fp32: max relative error <= 1e-5."""
+    spec = W.WORKLOADS["mlra4_f32_b1_h4_l256"]
+    inp = W.make_inputs(spec, "cuda")
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    compare_batch(inp, got)
+    # the absorbed query against the oracle's absorption
+    qa = oracle.absorb_query(inp.q_nope[0].cpu(), inp.w_uk.cpu())
+    check_close(got["q_abs"][0].double().numpy(), qa, "f32", "q_abs")
+
+
+@pytest.mark.parametrize("name,seqlens", [
+    ("mlra4_bf16_b16_h16_l4096_contig", [1, 63, 64, 65, 700, 1500]),
+    ("mlra4_bf16_b64_h32_l16384_paged", [129, 1000, 2049]),
+    ("mlra4_bf16_b128_h16_ragged1k_64k_paged", [1, 64, 333, 1024, 2500, 77]),
+])
+def test_bf16_oracle_sized(name, seqlens):
+    inp = _small(name, len(seqlens), seqlens)
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    compare_batch(inp, got)
+
+
+@pytest.mark.parametrize("name", ["mla_bf16_b8_h128_l131072_paged",
+                                  "mlra4_bf16_b8_h128_l131072_paged"])
+def test_bf16_h128_oracle_sized(name):
+    inp = _small(name, 2, [1100, 190])
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    compare_batch(inp, got, heads=[0, 1, 63, 100, 127])
+
+
+def test_empty_and_single_token_sequences():
+    inp = _small("mlra4_bf16_b64_h32_l16384_paged", 4, [0, 1, 0, 130])
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    assert torch.all(got["out"][0] == 0) and torch.all(got["out"][2] == 0)
+    assert torch.all(torch.isneginf(got["lse"][0]))
+    compare_batch(inp, got, seqs=[1, 3])
+
+
+def test_tail_rows_never_matter():
+    """Rows at or past seqlen hold NaN / huge values: the result must not change."""
+    inp = _small("mlra4_bf16_b16_h16_l4096_contig", 3, [100, 64, 190])
+    ref = run_gpu(inp)
+    inp.kv_cache[0, 100:] = float("nan")
+    inp.kv_cache[1, 64:] = 3.0e38
+    got = run_gpu(inp)
+    for k in ("out", "o_lat", "lse"):
+        assert torch.equal(got[k], ref[k]), k
+
+
+def test_paged_tail_rows_never_matter():
+    inp = _small("mlra4_bf16_b64_h32_l16384_paged", 2, [70, 5])
+    ref = run_gpu(inp)
+    flat = inp.kv_cache.view(-1, inp.spec.D)
+    pt = inp.page_table.cpu()
+    flat[int(pt[0, 1]) * 64 + 6: int(pt[0, 1]) * 64 + 64] = float("nan")
+    flat[int(pt[1, 0]) * 64 + 5: int(pt[1, 0]) * 64 + 64] = float("inf")
+    got = run_gpu(inp)
+    for k in ("out", "o_lat", "lse"):
+        assert torch.equal(got[k], ref[k]), k
+
+
+def test_page_permutation_invariance():
+    """Moving pages together with the page table leaves every output unchanged."""
+    inp = _small("mlra4_bf16_b128_h16_ragged1k_64k_paged", 3, [300, 1000, 65])
+    ref = run_gpu(inp)
+    n = inp.kv_cache.shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(5)).to("cuda")
+    new_cache = torch.empty_like(inp.kv_cache)
+    new_cache[perm] = inp.kv_cache
+    inp.page_table = torch.where(inp.page_table >= 0, perm[inp.page_table.clamp(min=0).long()].int(),
+                                 inp.page_table)
+    inp.kv_cache = new_cache
+    got = run_gpu(inp)
+    for k in ("out", "o_lat", "lse"):
+        torch.testing.assert_close(got[k], ref[k], rtol=0, atol=0)
+
+
+def test_ragged_isolation():
+    """A sequence's output does not depend on the other sequences in the batch
+    (nor on how the split planner cuts the batch)."""
+    big = _small("mlra4_bf16_b128_h16_ragged1k_64k_paged", 5, [3000, 17, 1200, 4100, 640])
+    one = W.DecodeInputs(spec=big.spec.replace(batch=1), seqlens=big.seqlens[3:4],
+                         q_nope=big.q_nope[3:4], q_rope=big.q_rope[3:4],
+                         w_uk=big.w_uk, w_uv=big.w_uv, kv_cache=big.kv_cache,
+                         page_table=big.page_table[3:4], max_len=big.max_len)
+    a = run_gpu(big)
+    b = run_gpu(one)
+    check_close(b["out"][0].double().numpy(), a["out"][3].double().numpy(), "f32", "isolation")
+
+
+def test_bad_page_sets_error_word():
+    inp = _small("mlra4_bf16_b64_h32_l16384_paged", 2, [200, 100])
+    inp.page_table[1, 0] = inp.kv_cache.shape[0] + 5
+    got = run_gpu(inp)
+    assert got["device_error"] == 6
+    ok = run_gpu(_small("mlra4_bf16_b64_h32_l16384_paged", 2, [200, 100]))
+    assert ok["device_error"] == 0
+
+
+def test_seqlen_beyond_capacity_sets_error_word():
+    inp = _small("mlra4_bf16_b16_h16_l4096_contig", 2, [100, 50])
+    inp.seqlens[0] = 10_000
+    got = run_gpu(inp)
+    assert got["device_error"] == 1
+
+
+def test_determinism():
+    inp = _small("mlra4_bf16_b64_h32_l16384_paged", 2, [2000, 999])
+    a = run_gpu(inp)
+    b = run_gpu(inp)
+    for k in ("out", "o_lat", "lse"):
+        assert torch.equal(a[k], b[k])
+
+
+# ---- full workload sizes, sampled outputs --------------------------------
+
+FULL = [
+    ("mlra4_bf16_b16_h16_l4096_contig", [(0, [0, 15]), (9, [7])]),
+    ("mlra4_bf16_b64_h32_l16384_paged", [(0, [0, 31]), (63, [5])]),
+    ("mlra4_bf16_b128_h16_ragged1k_64k_paged", [(5, [3]), (127, [0, 15])]),
+    ("mla_bf16_b8_h128_l131072_paged", [(0, [0, 127]), (7, [64])]),
+    ("mlra4_bf16_b8_h128_l131072_paged", [(0, [0, 127]), (7, [64])]),
+]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,samples", FULL)
+def test_full_size_sampled(name, samples):
+    spec = W.WORKLOADS[name]
+    inp = W.make_inputs(spec, "cuda")
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    assert torch.all(torch.isfinite(got["out"]))
+    L_all = inp.seqlens.cpu().numpy()
+    for seq, heads in samples:
+        ref = oracle.decode_sampled(spec, seq, heads, int(L_all[seq]))
+        check_close(got["out"][seq, heads].double().numpy(), ref.out[heads], spec.dtype,
+                    f"{name} seq {seq}")
+        check_close(got["o_lat"][seq, heads].double().numpy(), ref.o_lat[heads], spec.dtype,
+                    f"{name} seq {seq} o_lat")
