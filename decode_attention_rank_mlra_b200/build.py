@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmlra.so")
 SOURCES = ["mlra_api.cu", "k_small.cu", "k_decode_simt.cu", "k_decode_tc.cu"]
-HEADERS = ["mlra_internal.cuh", "../../include/mlra.h"]
+HEADERS = ["mlra_internal.cuh", "sm100_ptx.cuh", "../../include/mlra.h"]
 
 
 def nvcc_path() -> str:

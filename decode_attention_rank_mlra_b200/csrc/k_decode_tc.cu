@@ -1,11 +1,555 @@
-// Tensor-core decode kernel (tcgen05 / TMEM / TMA) -- not built yet.
+// Tensor-core split-KV decode attention over the bf16 latent cache (sm_100a).
+//
+// What it computes is the same as the SIMT kernel: for one split of one
+// sequence and every (head, branch) of the CTA's branch group,
+//   z_t = (q_abs . c_b[t] + q_rope . k_rope[t]) * scale,
+//   o = softmax(z) . c_b,  lse = log sum exp z
+// with one softmax per latent branch ("Multi-Head Low-Rank Attention",
+// Methodology, second paragraph) over the shared latent cache, the absorbed
+// "MQA-style" step of Main Findings ("three absorbable steps").
+//
+// How (one CTA per SM, persistent over a share of the tile stream):
+//  * warp 4 streams 64-token tiles of the cache with TMA (SWIZZLE_128B boxes of
+//    64 rows x 64 columns): the two boxes of each latent block c_b of the
+//    group and the RoPE box, into a multi-stage shared-memory ring;
+//  * warp 5 issues tcgen05.mma: S = Q . C^T (A = queries in TMEM, B = cache tile
+//    K-major) and O += P . C (A = probabilities in TMEM, B = the same tile,
+//    MN-major).  The 128 MMA rows are (branch, head, hi|lo): every head of the
+//    group is an M row, and per-branch MMAs write only their own rows through
+//    the disable-output-lane mask, so one tile in shared memory feeds every
+//    branch;
+//  * warps 0-3 (one per TMEM lane quadrant) run the online softmax of their
+//    rows and write P back into TMEM.
+// Precision: queries and probabilities are carried as bf16 hi + lo pairs (two
+// MMA rows per head), so both enter the fp32-accumulated products with about
+// 16 significant bits while the cache stays the bf16 it is stored as.
 #include "mlra_internal.cuh"
+#include "sm100_ptx.cuh"
+
+#include <cudaTypedefs.h>
+#include <math.h>
 
 namespace mlra {
-bool tc_supported(const mlra_config_t&) { return false; }
-void tc_grid(const mlra_config_t&, int num_sms, int* n_groups, int* ctas_per_group) {
-  *n_groups = 1;
-  *ctas_per_group = num_sms;
+namespace {
+
+using namespace ptx;
+
+constexpr int kBoxCols = 64;                 // bf16 columns per TMA box (128 B)
+constexpr int kBoxBytes = kTile * 128;       // 64 rows x 128 B
+constexpr int kThreadsTC = 192;              // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColQ = 0;                // q_abs rows (bf16 pairs): 64 columns
+constexpr uint32_t kColQr = 64;              // q_rope rows: 32 columns
+constexpr uint32_t kColS = 128;              // S / P double buffer: 2 x 64 columns
+constexpr uint32_t kColO = 256;              // O accumulator: 128 columns
+constexpr float kRescaleLog2 = 8.0f;         // rescale O only when the max grows by > 2^8
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kSmemLimit = 232448;           // max dynamic shared memory per block
+
+template <int G>
+struct TcShape {
+  static constexpr int kBoxes = 2 * G + 1;
+  static constexpr int kStage = kBoxes * kBoxBytes;
+  static constexpr int kStagesRaw = (kSmemLimit - 2048) / kStage;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kBars = 2 * kStages + 8;
+  static constexpr int kSmem = 1024 + kStages * kStage + kBars * 8 + 64;
+};
+
+struct Piece {
+  int s, t0, t1, slot, L;
+};
+
+struct Walker {
+  const int32_t* tile_off;
+  const int32_t* slot_off;
+  const int32_t* seqlens;
+  int batch, share, cap, gt, end;
+  __device__ bool next(Piece& p) {
+    if (gt >= end) return false;
+    const int s = find_seq(tile_off, batch, gt);
+    const int s0 = __ldg(tile_off + s), s1 = __ldg(tile_off + s + 1);
+    const int pe = min(end, s1);
+    p.s = s;
+    p.t0 = gt - s0;
+    p.t1 = pe - s0;
+    p.slot = __ldg(slot_off + s) + (gt / share - s0 / share);
+    p.L = min(max(__ldg(seqlens + s), 0), cap);
+    gt = pe;
+    return true;
+  }
+};
+
+// Bounded mbarrier wait: false on timeout (error recorded) or when another role aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      set_error(err, MLRA_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
 }
-cudaError_t launch_decode_tc(const DecodeArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int G, int HPC>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+  using S = TcShape<G>;
+  constexpr int NST = S::kStages;
+  constexpr int STAGE = S::kStage;
+  constexpr int WPB = HPC / 16;  // softmax warps per branch
+  static_assert(G * WPB <= 4, "rows exceed 128");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NST * STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t bar0 = smem_addr(bars);
+  auto FULL = [&](int i) { return bar0 + 8u * i; };
+  auto EMPTY = [&](int i) { return bar0 + 8u * (NST + i); };
+  auto SFULL = [&](int i) { return bar0 + 8u * (2 * NST + i); };
+  auto PREADY = [&](int i) { return bar0 + 8u * (2 * NST + 2 + i); };
+  // PV of tile k commits to PVDONE(k & 1): a waiter for PV(k) has always seen
+  // S(k) or later, which implies PV(k-2) is complete, so parity waits are exact.
+  auto PVDONE = [&](int i) { return bar0 + 8u * (2 * NST + 4 + i); };
+  const uint32_t QREADY = bar0 + 8u * (2 * NST + 6);
+  const uint32_t DRAIN = bar0 + 8u * (2 * NST + 7);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
+  int32_t* err = &hdr->error;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(FULL(i), 1);
+      mbar_init(EMPTY(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(SFULL(i), 1);
+      mbar_init(PREADY(i), 4);
+    }
+    mbar_init(PVDONE(0), 1);
+    mbar_init(PVDONE(1), 1);
+    mbar_init(QREADY, 4);
+    mbar_init(DRAIN, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const char* wsc = static_cast<const char*>(a.ws);
+  const int nb = a.cfg.n_blocks, H = a.cfg.n_heads;
+  const int g = blockIdx.x / a.ctas_per_group;
+  const int c = blockIdx.x % a.ctas_per_group;
+  const int total = hdr->total_tiles, share = hdr->share;
+  Walker walk{reinterpret_cast<const int32_t*>(wsc + a.L.tile_off),
+              reinterpret_cast<const int32_t*>(wsc + a.L.slot_off),
+              a.seqlens, a.batch, share, a.cap, c * share, min(total, (c + 1) * share)};
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap);
+      Piece p;
+      int it = 0;
+      bool ok = true;
+      while (ok && walk.next(p)) {
+        for (int t = p.t0; t < p.t1; ++t, ++it) {
+          const int st = it % NST;
+          if (!wait_bar(EMPTY(st), ((it / NST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          int row;
+          if (a.page_table) {
+            const int pg = __ldg(a.page_table + size_t(p.s) * a.max_pages + t);
+            if (pg < 0 || pg >= a.num_pages) {
+              set_error(err, MLRA_ERR_BAD_PAGE);
+              row = -2 * kTile;  // out of bounds: the box is zero-filled
+            } else {
+              row = pg * kPageSize;
+            }
+          } else {
+            row = p.s * a.max_pages + t * kTile;
+          }
+          mbar_arrive_expect_tx(FULL(st), STAGE);
+          const uint32_t dst = smem_addr(stages + st * STAGE);
+#pragma unroll
+          for (int bx = 0; bx < G; ++bx) {
+            const int br = g * G + bx;
+            tma_load_2d(dst + (2 * bx) * kBoxBytes, &tmap, br * 128, row, FULL(st));
+            tma_load_2d(dst + (2 * bx + 1) * kBoxBytes, &tmap, br * 128 + kBoxCols, row, FULL(st));
+          }
+          tma_load_2d(dst + 2 * G * kBoxBytes, &tmap, nb * 128, row, FULL(st));
+        }
+      }
+      if (!ok) {
+        // let loads already in flight land before the CTA can exit
+        for (int j = 0; j < NST; ++j) {
+          const int k = it - 1 - j;
+          if (k < 0) break;
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(FULL(k % NST), (k / NST) & 1) && globaltimer() - t0 < 10000000ull) {}
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kTile, false, false);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
+    uint32_t mask[G][4];
+#pragma unroll
+    for (int bx = 0; bx < G; ++bx)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) mask[bx][w] = (w / WPB == bx) ? 0u : 0xFFFFFFFFu;
+    Piece p;
+    int it = 0, piece = 0;
+    bool ok = true;
+    auto issue_pv = [&](int pit, bool first) {
+      const int pst = pit % NST, psb = pit & 1;
+      const uint32_t sbase = smem_addr(stages + pst * STAGE);
+      if (lane == 0) {
+#pragma unroll
+        for (int bx = 0; bx < G; ++bx) {
+          if (g * G + bx >= nb) continue;
+#pragma unroll
+          for (int k = 0; k < kTile / 16; ++k) {
+            const uint64_t bd = smem_desc(sbase + (2 * bx) * kBoxBytes + k * 16 * 128, kBoxBytes,
+                                          1024, kSwizzle128B);
+            mma_ts(tmem + kColO, tmem + kColS + 64 * psb + 8 * k, bd, kIdescPV,
+                   (first && k == 0) ? 0u : 1u, mask[bx][0], mask[bx][1], mask[bx][2],
+                   mask[bx][3]);
+          }
+        }
+        mma_commit(EMPTY(pst));
+        mma_commit(PVDONE(pit & 1));
+      }
+      __syncwarp();
+    };
+    while (ok && walk.next(p)) {
+      if (!wait_bar(QREADY, piece & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      const int first_it = it;
+      for (int t = p.t0; t < p.t1; ++t, ++it) {
+        const int st = it % NST, sb = it & 1;
+        if (!wait_bar(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
+        const int valid = min(kTile, p.L - t * kTile);
+        if (valid < kTile) {
+          // zero the rows past the sequence end (whatever the cache holds there)
+          const int per_box = (kTile - valid) * 8;
+          uint8_t* sp = stages + st * STAGE;
+          for (int i = lane; i < per_box * S::kBoxes; i += 32) {
+            const int bx = i / per_box, rem = i % per_box;
+            *reinterpret_cast<uint4*>(sp + bx * kBoxBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sbase = smem_addr(stages + st * STAGE);
+          const uint32_t d = tmem + kColS + 64 * sb;
+#pragma unroll
+          for (int bx = 0; bx < G; ++bx) {
+            if (g * G + bx >= nb) continue;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint64_t bd = smem_desc(sbase + (2 * bx + (k >> 2)) * kBoxBytes + (k & 3) * 32,
+                                            16, 1024, kSwizzle128B);
+              mma_ts(d, tmem + kColQ + 8 * k, bd, kIdescQK, k > 0 ? 1u : 0u, mask[bx][0],
+                     mask[bx][1], mask[bx][2], mask[bx][3]);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t bd = smem_desc(sbase + 2 * G * kBoxBytes + k * 32, 16, 1024, kSwizzle128B);
+            mma_ts(d, tmem + kColQr + 8 * k, bd, kIdescQK, 1u, 0u, 0u, 0u, 0u);
+          }
+          mma_commit(SFULL(sb));
+        }
+        __syncwarp();
+        if (it > first_it) {
+          const int pit = it - 1;
+          if (!wait_bar(PREADY(pit & 1), (pit >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(pit, pit == first_it);
+        }
+      }
+      if (!ok) break;
+      const int pit = it - 1;
+      if (!wait_bar(PREADY(pit & 1), (pit >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      issue_pv(pit, pit == first_it);
+      ++piece;
+    }
+    if (!ok && lane == 0) {
+      // drain MMAs already issued before TMEM is released
+      mma_commit(DRAIN);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(DRAIN, 0) && globaltimer() - t0 < 10000000ull) {}
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps 0-3
+    const int bg = warp / WPB;
+    const int branch = g * G + bg;
+    const bool active = bg < G && branch < nb;
+    const int x = lane >> 4;                         // 0: hi row, 1: lo row
+    const int head = 16 * (warp % WPB) + (lane & 15);
+    const uint32_t row_t = tmem + (uint32_t(32 * warp) << 16);
+    const float sl2 = a.cfg.softmax_scale * 1.4426950408889634f;
+    float* o_part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + a.L.o_part);
+    float* lse_part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + a.L.lse_part);
+    const __nv_bfloat16* q_rope = static_cast<const __nv_bfloat16*>(a.q_rope);
+    Piece p;
+    int it = 0, piece = 0;
+    bool ok = true;
+    while (ok && walk.next(p)) {
+      // ---- this piece's queries into TMEM (A operand rows)
+      {
+        uint32_t r[32];
+        const float* q = a.q_abs + ((size_t(p.s) * H + head) * nb + branch) * 128;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float v0 = 0.f, v1 = 0.f;
+            if (active) {
+              v0 = __ldg(q + 64 * half + 2 * j);
+              v1 = __ldg(q + 64 * half + 2 * j + 1);
+              if (x) {  // lo part: what the bf16 hi part leaves out
+                v0 -= __bfloat162float(__float2bfloat16_rn(v0));
+                v1 -= __bfloat162float(__float2bfloat16_rn(v1));
+              }
+            }
+            r[j] = pack_bf16(v0, v1);
+          }
+          tmem_st32(row_t + kColQ + 32 * half, r);
+        }
+        const unsigned short* qr =
+            reinterpret_cast<const unsigned short*>(q_rope + (size_t(p.s) * H + head) * 64);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          r[j] = (active && x == 0) ? (uint32_t(__ldg(qr + 2 * j)) | (uint32_t(__ldg(qr + 2 * j + 1)) << 16))
+                                    : 0u;
+        tmem_st32(row_t + kColQr, r);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(QREADY);
+      }
+      float m = -INFINITY, l = 0.f;
+      for (int t = p.t0; t < p.t1; ++t, ++it) {
+        const int sb = it & 1;
+        if (!wait_bar(SFULL(sb), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[64];
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(row_t + kColS + 64 * sb, r0);
+          tmem_ld32(row_t + kColS + 64 * sb + 32, r1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) { v[k] = r0[k]; v[32 + k] = r1[k]; }
+        }
+        const int valid = min(kTile, p.L - t * kTile);
+        float s[32];
+        float mt = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float send = __uint_as_float(x ? v[k] : v[32 + k]);
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+          const float own = __uint_as_float(x ? v[32 + k] : v[k]);
+          const int tok = 32 * x + k;
+          s[k] = (tok < valid) ? (own + recv) * sl2 : -INFINITY;
+          mt = fmaxf(mt, s[k]);
+        }
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+        if (t == p.t0) {
+          m = mt;
+        } else if (mt > m + kRescaleLog2) {
+          const float alpha = exp2f(m - mt);
+          m = mt;
+          l *= alpha;
+          // O must not be in use by the previous PV while it is rescaled
+          const int pk = it - 1;
+          if (!wait_bar(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(row_t + kColO + 32 * ch, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+            tmem_st32(row_t + kColO + 32 * ch, r);
+          }
+          tmem_wait_st();
+        }
+        float ls = 0.f;
+        uint32_t whi[16], wlo[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float p0 = exp2f(s[k] - m), p1 = exp2f(s[k + 1] - m);
+          ls += p0 + p1;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          const float2 hf = __bfloat1622float2(h2);
+          whi[k / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          wlo[k / 2] = pack_bf16(p0 - hf.x, p1 - hf.y);
+        }
+        l += ls;
+        uint32_t prow[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t recv = __shfl_xor_sync(0xffffffffu, x ? whi[j] : wlo[j], 16);
+          prow[j] = x ? recv : whi[j];
+          prow[16 + j] = x ? wlo[j] : recv;
+        }
+        tmem_st32(row_t + kColS + 64 * sb, prow);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(PREADY(sb));
+      }
+      if (!ok) break;
+      // ---- epilogue: o = (O_hi + O_lo) / l, lse
+      {
+        const int pk = it - 1;
+        if (!wait_bar(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      }
+      tc_fence_after();
+      const float l_tot = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      float* dst = o_part + ((size_t(p.slot) * H + head) * nb + branch) * 128;
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(row_t + kColO + 32 * j, ra);
+        tmem_ld32(row_t + kColO + 64 + 32 * j, rb);
+        tmem_wait_ld();
+        float o[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float send = __uint_as_float(x ? ra[k] : rb[k]);
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+          o[k] = (__uint_as_float(x ? rb[k] : ra[k]) + recv) * inv;
+        }
+        if (active) {
+          float4* d4 = reinterpret_cast<float4*>(dst + 64 * x + 32 * j);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) d4[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        }
+      }
+      if (active && x == 0)
+        lse_part[(size_t(p.slot) * H + head) * nb + branch] =
+            l_tot > 0.f ? (m + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
+      ++piece;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int g_of(const mlra_config_t& c) {
+  const int per = 64 / c.n_heads;
+  return c.n_blocks < per ? c.n_blocks : per;
+}
+
+template <int G, int HPC>
+cudaError_t launch_t(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st) {
+  using S = TcShape<G>;
+  auto kern = decode_tc_kernel<G, HPC>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  kern<<<a.n_groups * a.ctas_per_group, kThreadsTC, S::kSmem, st>>>(map, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(const mlra_config_t& c) {
+  if (c.dtype != MLRA_BF16 || c.d_cb != 128 || c.d_r != 64) return false;
+  if (c.n_heads != 16 && c.n_heads != 32 && c.n_heads != 64) return false;
+  if (c.n_blocks != 1 && c.n_blocks != 2 && c.n_blocks != 4) return false;
+  return c.n_blocks % g_of(c) == 0;
+}
+
+void tc_grid(const mlra_config_t& c, int num_sms, int* n_groups, int* ctas_per_group) {
+  *n_groups = c.n_blocks / g_of(c);
+  *ctas_per_group = num_sms / *n_groups > 0 ? num_sms / *n_groups : 1;
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
+  const mlra_config_t& c = a.cfg;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const int D = c.n_blocks * c.d_cb + c.d_r;
+  const uint64_t rows = a.page_table ? uint64_t(a.num_pages) * kPageSize
+                                     : uint64_t(a.batch) * uint64_t(a.max_pages);
+  if (rows >= (uint64_t(1) << 31)) return cudaErrorInvalidValue;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+  cuuint32_t box[2] = {kBoxCols, kTile};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.kv_cache), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const int G = g_of(c);
+  switch (c.n_heads * 10 + G) {
+    case 164: return launch_t<4, 16>(map, a, st);
+    case 162: return launch_t<2, 16>(map, a, st);
+    case 161: return launch_t<1, 16>(map, a, st);
+    case 322: return launch_t<2, 32>(map, a, st);
+    case 321: return launch_t<1, 32>(map, a, st);
+    case 641: return launch_t<1, 64>(map, a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace mlra
