@@ -37,7 +37,7 @@ STATUS = {
 EXPORTS = [
     "mlra_status_string", "mlra_version", "mlra_absorb_q", "mlra_workspace_size",
     "mlra_decode_attn", "mlra_splitkv_combine", "mlra_out_proj", "mlra_get_device_error",
-    "mlra_decode_kernel_kind",
+    "mlra_decode_kernel_kind", "mlra_decode_attn_noalloc",
 ]
 
 
@@ -101,6 +101,7 @@ def lib() -> ctypes.CDLL:
         "mlra_out_proj": (I32, [CP, P, P, P, I32, P]),
         "mlra_get_device_error": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "mlra_decode_kernel_kind": (I32, [CP]),
+        "mlra_decode_attn_noalloc": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -223,6 +224,41 @@ def out_proj(cfg: Config, o_latent: torch.Tensor, w_uv: torch.Tensor,
     return out
 
 
+def decode_attn_noalloc(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor,
+                        kv_cache: torch.Tensor, page_table: Optional[torch.Tensor],
+                        seqlens: torch.Tensor, max_pages: int, o_latent: torch.Tensor,
+                        lse: Optional[torch.Tensor] = None,
+                        device_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Steps 2a + 2b with the library's own fixed scratch (no workspace).
+
+    For callers that cannot allocate device memory (a plugin whose host owns
+    the device allocator, or a server that reserved all free HBM up front):
+    nothing is allocated here or in the library.  All calls share one 16 MiB
+    array inside libmlra.so, so calls that overlap on the GPU race; batches
+    needing more scratch are rejected with MLRA_ERR_WORKSPACE.  Outputs as
+    ``splitkv_combine``; ``device_status`` (one int32 on the device) receives
+    the call's device error word.
+    """
+    _need(q_abs, "q_abs", torch.float32)
+    _need(q_rope, "q_rope", cfg.torch_dtype)
+    _need(kv_cache, "kv_cache", cfg.torch_dtype)
+    _need(seqlens, "seqlens", torch.int32)
+    _need(o_latent, "o_latent", torch.float32)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    if device_status is not None:
+        _need(device_status, "device_status", torch.int32)
+    num_pages = 0
+    if page_table is not None:
+        _need(page_table, "page_table", torch.int32)
+        num_pages = kv_cache.shape[0]
+    B = seqlens.shape[0]
+    _check("mlra_decode_attn_noalloc", lib().mlra_decode_attn_noalloc(
+        ctypes.byref(cfg), _ptr(q_abs), _ptr(q_rope), _ptr(kv_cache), num_pages, _ptr(page_table),
+        int(max_pages), _ptr(seqlens), B, _ptr(o_latent), _ptr(lse), _ptr(device_status),
+        _stream(stream)))
+
+
 def get_device_error(workspace: torch.Tensor, stream=None) -> int:
     """Device-side status recorded in the workspace (synchronises the stream)."""
     v = ctypes.c_int32(0)
@@ -270,5 +306,6 @@ class Decoder:
 __all__ = [
     "Config", "make_config", "lib", "absorb_q", "workspace_size", "alloc_workspace",
     "decode_attn", "splitkv_combine", "out_proj", "get_device_error", "decode_kernel_kind",
+    "decode_attn_noalloc",
     "Decoder", "MlraError", "EXPORTS", "F32", "BF16",
 ]

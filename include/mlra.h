@@ -177,6 +177,37 @@ MLRA_API mlra_status_t mlra_get_device_error(const void* workspace, size_t works
                                     int32_t* device_status, mlra_stream_t stream);
 
 /*
+ * Steps 2a + 2b without a caller workspace (no counterpart in the paper: this
+ * is a deployment convenience of the library).
+ * Some callers cannot call cudaMalloc: a plugin running inside a host
+ * framework that owns all device memory through its own allocator, or a
+ * serving process that reserves all free HBM for the KV cache at start-up and
+ * must not allocate later (cudaMalloc may also synchronise the device, which a
+ * latency-bound decode loop cannot afford).  This call needs no workspace and
+ * allocates nothing: its scratch (split plan, split partials, error word) is a
+ * fixed 16 MiB array inside libmlra.so, held on every GPU that loads the
+ * library until the process exits.
+ *   Arguments as mlra_decode_attn, then as mlra_splitkv_combine:
+ *   o_latent      : [batch, n_heads, n_blocks, d_cb] fp32 (written)
+ *   lse           : [batch, n_heads, n_blocks] fp32 (written; may be NULL)
+ *   device_status : one int32 in device memory (may be NULL); receives the
+ *                   device error word of this call (MLRA_OK, MLRA_ERR_BAD_PAGE,
+ *                   MLRA_ERR_TIMEOUT, MLRA_ERR_INVALID_ARG for clamped seqlens)
+ * Returns MLRA_ERR_WORKSPACE, launching nothing, when the scratch this batch
+ * needs (mlra_workspace_size) exceeds 16 MiB.  The first call on a device looks
+ * up the array's device address with that device current; make that first
+ * call before capturing any stream.  All calls share the one array and it
+ * keeps the last call's contents: calls ordered on one stream are safe, calls
+ * that overlap on the GPU (other streams, other host threads) race on it.
+ */
+MLRA_API mlra_status_t mlra_decode_attn_noalloc(const mlra_config_t* cfg, const float* q_abs,
+                                                const void* q_rope, const void* kv_cache,
+                                                int64_t num_pages, const int32_t* page_table,
+                                                int32_t max_pages, const int32_t* seqlens,
+                                                int32_t batch, float* o_latent, float* lse,
+                                                int32_t* device_status, mlra_stream_t stream);
+
+/*
  * Which decode kernel mlra_decode_attn would launch for cfg on the current
  * device: 1 = tensor-core kernel (tcgen05 / TMEM / TMA), 2 = fp32 SIMT kernel,
  * 0 = unsupported.  Host-only query, launches nothing.
