@@ -275,6 +275,40 @@ def run_ours(args):
         kev[i][1].record(stream)
     torch.cuda.synchronize()
     k_ms = [a.elapsed_time(b) for a, b in kev]
+    # ---- per-call breakdown: each call captured alone in a CUDA graph and
+    # replayed back to back, one event pair around all replays -----------------
+    calls = {
+        "absorb_q": lambda i: mlra.absorb_q(cfg, inp.q_nope, inp.w_uk, dec.q_abs),
+        "decode_attn": lambda i: mlra.decode_attn(cfg, dec.q_abs, inp.q_rope, caches[i % copies],
+                                                  inp.page_table, inp.seqlens, max_pages,
+                                                  dec.workspace),
+        "splitkv_combine": lambda i: mlra.splitkv_combine(cfg, dec.workspace, B, dec.o_latent,
+                                                          dec.lse),
+        "out_proj": lambda i: mlra.out_proj(cfg, dec.o_latent, inp.w_uv, dec.out),
+    }
+    breakdown = {}
+    reps = max(10, min(args.steps, 200))
+    for name, fn in calls.items():
+        gs = []
+        with torch.cuda.stream(side):
+            for i in range(copies):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    fn(i)
+                gs.append(g)
+        stream.wait_stream(side)
+        for i in range(2 * copies):
+            gs[i % copies].replay()
+        torch.cuda.synchronize()
+        b0 = torch.cuda.Event(enable_timing=True)
+        b1 = torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for i in range(reps):
+            gs[i % copies].replay()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        breakdown[name] = b0.elapsed_time(b1) * 1e3 / reps
+        del gs
     # ---- end-to-end: host buffers, copies inside the timed region ------------
     h_qn = inp.q_nope.cpu().pin_memory()
     h_qr = inp.q_rope.cpu().pin_memory()
@@ -348,6 +382,7 @@ def run_ours(args):
                     "note": "queries and seqlens copied in, output copied out every step; "
                             "the KV cache is device-resident state"},
             "clocks": clocks,
+            "breakdown_us": breakdown,
             "gpu_launches": 5 * args.steps,
             "timing": "K replays of a CUDA graph of the whole step (5 kernels), one event pair around all K",
         }

@@ -42,7 +42,9 @@ constexpr uint32_t kColQ = 0;                // q_abs rows (bf16 pairs): 64 colu
 constexpr uint32_t kColQr = 64;              // q_rope rows: 32 columns
 constexpr uint32_t kColS = 128;              // S / P double buffer: 2 x 64 columns
 constexpr uint32_t kColO = 256;              // O accumulator: 128 columns
-constexpr float kRescaleLog2 = 8.0f;         // rescale O only when the max grows by > 2^8
+// A row keeps its running max until a tile exceeds it by 2^8; the O rescale that
+// follows is done by the row's own thread on its own TMEM lane.
+constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kSmemLimit = 232448;           // max dynamic shared memory per block
 
@@ -54,20 +56,31 @@ struct TcShape {
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kBars = 2 * kStages + 8;
   static constexpr int kSmem = 1024 + kStages * kStage + kBars * 8 + 64;
+  static_assert(kStages >= 3, "too few pipeline stages");
 };
 
 struct Piece {
   int s, t0, t1, slot, L;
 };
 
+// Walks the pieces (sequence, tile range) of one CTA's share of the tile stream.
+// Only the first piece needs a search; the next ones follow sequence by sequence.
 struct Walker {
   const int32_t* tile_off;
   const int32_t* slot_off;
   const int32_t* seqlens;
   int batch, share, cap, gt, end;
+  int cur = -1;
   __device__ bool next(Piece& p) {
     if (gt >= end) return false;
-    const int s = find_seq(tile_off, batch, gt);
+    int s;
+    if (cur < 0) {
+      s = find_seq(tile_off, batch, gt);
+    } else {
+      s = cur + 1;
+      while (__ldg(tile_off + s + 1) <= gt) ++s;  // skip empty sequences
+    }
+    cur = s;
     const int s0 = __ldg(tile_off + s), s1 = __ldg(tile_off + s + 1);
     const int pe = min(end, s1);
     p.s = s;
@@ -103,13 +116,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// G branches x HPC heads per CTA (rows = G * HPC * 2 <= 128).  The grid is
+// (branch groups x head groups) x CTAs per group; one CTA per SM.
 template <int G, int HPC>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   using S = TcShape<G>;
   constexpr int NST = S::kStages;
   constexpr int STAGE = S::kStage;
-  constexpr int WPB = HPC / 16;  // softmax warps per branch
+  constexpr int WPB = HPC / 16;  // TMEM lane quadrants per branch
   static_assert(G * WPB <= 4, "rows exceed 128");
 
   extern __shared__ uint8_t smem_raw[];
@@ -142,9 +157,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(SFULL(i), 1);
       mbar_init(PREADY(i), 4);
+      mbar_init(PVDONE(i), 1);
     }
-    mbar_init(PVDONE(0), 1);
-    mbar_init(PVDONE(1), 1);
     mbar_init(QREADY, 4);
     mbar_init(DRAIN, 1);
     *abort_flag = 0;
@@ -161,8 +175,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   const char* wsc = static_cast<const char*>(a.ws);
   const int nb = a.cfg.n_blocks, H = a.cfg.n_heads;
-  const int g = blockIdx.x / a.ctas_per_group;
+  const int grp = blockIdx.x / a.ctas_per_group;
   const int c = blockIdx.x % a.ctas_per_group;
+  const int g = grp % (nb / G);            // branch group
+  const int head0 = (grp / (nb / G)) * HPC;  // first head of this CTA's head group
   const int total = hdr->total_tiles, share = hdr->share;
   Walker walk{reinterpret_cast<const int32_t*>(wsc + a.L.tile_off),
               reinterpret_cast<const int32_t*>(wsc + a.L.slot_off),
@@ -172,6 +188,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tensormap(&tmap);
+      const uint64_t evict_first = policy_evict_first();  // the cache is streamed once
       Piece p;
       int it = 0;
       bool ok = true;
@@ -196,10 +213,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
           for (int bx = 0; bx < G; ++bx) {
             const int br = g * G + bx;
-            tma_load_2d(dst + (2 * bx) * kBoxBytes, &tmap, br * 128, row, FULL(st));
-            tma_load_2d(dst + (2 * bx + 1) * kBoxBytes, &tmap, br * 128 + kBoxCols, row, FULL(st));
+            tma_load_2d_hint(dst + (2 * bx) * kBoxBytes, &tmap, br * 128, row, FULL(st), evict_first);
+            tma_load_2d_hint(dst + (2 * bx + 1) * kBoxBytes, &tmap, br * 128 + kBoxCols, row,
+                             FULL(st), evict_first);
           }
-          tma_load_2d(dst + 2 * G * kBoxBytes, &tmap, nb * 128, row, FULL(st));
+          tma_load_2d_hint(dst + 2 * G * kBoxBytes, &tmap, nb * 128, row, FULL(st), evict_first);
         }
       }
       if (!ok) {
@@ -214,41 +232,43 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop; each MMA / commit is issued by one elected
+    // lane with warp-uniform operands (compile-time offsets from per-stage
+    // descriptors), which keeps the issue rate at the tensor core's pace.
+    //  QK : S[rows, tokens] = Q[rows, K] . C[tokens, K]^T  (A: TMEM, B: smem K-major)
+    //  PV : O[rows, features] += P[rows, tokens] . C_b[tokens, features]
+    //       (A: probabilities in TMEM over the S buffer, B: the same tile, MN-major)
+    // Rows of other branches are kept out of each branch's MMAs by the
+    // disable-output-lane mask.
     constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kTile, false, false);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
-    uint32_t mask[G][4];
-#pragma unroll
-    for (int bx = 0; bx < G; ++bx)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) mask[bx][w] = (w / WPB == bx) ? 0u : 0xFFFFFFFFu;
+    const uint32_t sbase0 = smem_addr(stages);
+    const uint64_t dK = smem_desc(sbase0, 16, 1024, kSwizzle128B);
+    const uint64_t dMN = smem_desc(sbase0, kBoxBytes, 1024, kSwizzle128B);
     Piece p;
     int it = 0, piece = 0;
+    int prev = -1;            // tile whose PV is still to be issued
+    bool prev_first = false;  // ...and whether it opens its piece
     bool ok = true;
     auto issue_pv = [&](int pit, bool first) {
-      const int pst = pit % NST, psb = pit & 1;
-      const uint32_t sbase = smem_addr(stages + pst * STAGE);
-      if (lane == 0) {
+      const uint64_t d = dMN + uint64_t(((pit % NST) * STAGE) >> 4);
+      const uint32_t a_p = tmem + kColS + 64 * (pit & 1);
 #pragma unroll
-        for (int bx = 0; bx < G; ++bx) {
-          if (g * G + bx >= nb) continue;
+      for (int bx = 0; bx < G; ++bx) {
+        if (g * G + bx >= nb) continue;
 #pragma unroll
-          for (int k = 0; k < kTile / 16; ++k) {
-            const uint64_t bd = smem_desc(sbase + (2 * bx) * kBoxBytes + k * 16 * 128, kBoxBytes,
-                                          1024, kSwizzle128B);
-            mma_ts(tmem + kColO, tmem + kColS + 64 * psb + 8 * k, bd, kIdescPV,
-                   (first && k == 0) ? 0u : 1u, mask[bx][0], mask[bx][1], mask[bx][2],
-                   mask[bx][3]);
-          }
-        }
-        mma_commit(EMPTY(pst));
-        mma_commit(PVDONE(pit & 1));
+        for (int k = 0; k < kTile / 16; ++k)
+          mma_ts_warp(tmem + kColO, a_p + 8 * k,
+                      d + uint64_t((2 * bx * kBoxBytes + k * 16 * 128) >> 4), kIdescPV,
+                      (first && k == 0) ? 0u : 1u, (0 / WPB == bx) ? 0u : ~0u,
+                      (1 / WPB == bx) ? 0u : ~0u, (2 / WPB == bx) ? 0u : ~0u,
+                      (3 / WPB == bx) ? 0u : ~0u);
       }
-      __syncwarp();
+      mma_commit_warp(EMPTY(pit % NST));
+      mma_commit_warp(PVDONE(pit & 1));
     };
     while (ok && walk.next(p)) {
       if (!wait_bar(QREADY, piece & 1, abort_flag, err)) { ok = false; break; }
-      tc_fence_after();
-      const int first_it = it;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int st = it % NST, sb = it & 1;
         if (!wait_bar(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
@@ -263,101 +283,125 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                 make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
-          __syncwarp();
         }
+        __syncwarp();
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sbase = smem_addr(stages + st * STAGE);
-          const uint32_t d = tmem + kColS + 64 * sb;
+        {
+          const uint64_t d = dK + uint64_t((st * STAGE) >> 4);
+          const uint32_t s_acc = tmem + kColS + 64 * sb;
 #pragma unroll
           for (int bx = 0; bx < G; ++bx) {
             if (g * G + bx >= nb) continue;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint64_t bd = smem_desc(sbase + (2 * bx + (k >> 2)) * kBoxBytes + (k & 3) * 32,
-                                            16, 1024, kSwizzle128B);
-              mma_ts(d, tmem + kColQ + 8 * k, bd, kIdescQK, k > 0 ? 1u : 0u, mask[bx][0],
-                     mask[bx][1], mask[bx][2], mask[bx][3]);
-            }
+            for (int k = 0; k < 8; ++k)
+              mma_ts_warp(s_acc, tmem + kColQ + 8 * k,
+                          d + uint64_t(((2 * bx + (k >> 2)) * kBoxBytes + (k & 3) * 32) >> 4),
+                          kIdescQK, k > 0 ? 1u : 0u, (0 / WPB == bx) ? 0u : ~0u,
+                          (1 / WPB == bx) ? 0u : ~0u, (2 / WPB == bx) ? 0u : ~0u,
+                          (3 / WPB == bx) ? 0u : ~0u);
           }
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t bd = smem_desc(sbase + 2 * G * kBoxBytes + k * 32, 16, 1024, kSwizzle128B);
-            mma_ts(d, tmem + kColQr + 8 * k, bd, kIdescQK, 1u, 0u, 0u, 0u, 0u);
-          }
-          mma_commit(SFULL(sb));
+          for (int k = 0; k < 4; ++k)
+            mma_ts_warp(s_acc, tmem + kColQr + 8 * k,
+                        d + uint64_t((2 * G * kBoxBytes + k * 32) >> 4), kIdescQK, 1u, 0u, 0u, 0u,
+                        0u);
+          mma_commit_warp(SFULL(sb));
         }
-        __syncwarp();
-        if (it > first_it) {
-          const int pit = it - 1;
-          if (!wait_bar(PREADY(pit & 1), (pit >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (prev >= 0) {
+          if (!wait_bar(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(pit, pit == first_it);
+          issue_pv(prev, prev_first);
         }
+        prev = it;
+        prev_first = (t == p.t0);
       }
-      if (!ok) break;
-      const int pit = it - 1;
-      if (!wait_bar(PREADY(pit & 1), (pit >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      tc_fence_after();
-      issue_pv(pit, pit == first_it);
       ++piece;
     }
-    if (!ok && lane == 0) {
+    if (ok && prev >= 0) {
+      if (wait_bar(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) {
+        tc_fence_after();
+        issue_pv(prev, prev_first);
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok) {
       // drain MMAs already issued before TMEM is released
-      mma_commit(DRAIN);
+      mma_commit_warp(DRAIN);
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(DRAIN, 0) && globaltimer() - t0 < 10000000ull) {}
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warps 0-3
+    // Thread = one row (TMEM lane): branch bg, head, hi (x=0) or lo (x=1) part.
+    // The hi and lo rows of a head sit 16 lanes apart and trade halves with
+    // shuffles; every other step is the thread's own.
     const int bg = warp / WPB;
     const int branch = g * G + bg;
     const bool active = bg < G && branch < nb;
-    const int x = lane >> 4;                         // 0: hi row, 1: lo row
-    const int head = 16 * (warp % WPB) + (lane & 15);
+    const int x = lane >> 4;                                 // 0: hi row, 1: lo row
+    const int head = head0 + 16 * (warp % WPB) + (lane & 15);
     const uint32_t row_t = tmem + (uint32_t(32 * warp) << 16);
     const float sl2 = a.cfg.softmax_scale * 1.4426950408889634f;
     float* o_part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + a.L.o_part);
     float* lse_part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + a.L.lse_part);
-    const __nv_bfloat16* q_rope = static_cast<const __nv_bfloat16*>(a.q_rope);
-    Piece p;
-    int it = 0, piece = 0;
-    bool ok = true;
-    while (ok && walk.next(p)) {
-      // ---- this piece's queries into TMEM (A operand rows)
-      {
-        uint32_t r[32];
-        const float* q = a.q_abs + ((size_t(p.s) * H + head) * nb + branch) * 128;
+    const unsigned short* q_rope = static_cast<const unsigned short*>(a.q_rope);
+    // (q_abs rows are 512 B and q_rope rows 128 B apart; both bases are 16-byte
+    // aligned, so whole rows are read with 16-byte loads.)
+    auto q_row = [&](const Piece& pc) {
+      return reinterpret_cast<const float4*>(a.q_abs + ((size_t(pc.s) * H + head) * nb + branch) * 128);
+    };
+    auto qr_row = [&](const Piece& pc) {
+      return reinterpret_cast<const uint4*>(q_rope + (size_t(pc.s) * H + head) * 64);
+    };
+    auto write_q = [&](const Piece& pc) {
+      uint32_t r[32];
+      const float4* q = q_row(pc);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < 2; ++half) {
+        float4 f[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float v0 = 0.f, v1 = 0.f;
-            if (active) {
-              v0 = __ldg(q + 64 * half + 2 * j);
-              v1 = __ldg(q + 64 * half + 2 * j + 1);
-              if (x) {  // lo part: what the bf16 hi part leaves out
-                v0 -= __bfloat162float(__float2bfloat16_rn(v0));
-                v1 -= __bfloat162float(__float2bfloat16_rn(v1));
-              }
-            }
-            r[j] = pack_bf16(v0, v1);
+        for (int j = 0; j < 16; ++j) f[j] = active ? __ldg(q + 16 * half + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float v[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
+          if (x) {  // lo part: what the bf16 hi part leaves out
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] -= __bfloat162float(__float2bfloat16_rn(v[e]));
           }
-          tmem_st32(row_t + kColQ + 32 * half, r);
+          r[2 * j] = pack_bf16(v[0], v[1]);
+          r[2 * j + 1] = pack_bf16(v[2], v[3]);
         }
-        const unsigned short* qr =
-            reinterpret_cast<const unsigned short*>(q_rope + (size_t(p.s) * H + head) * 64);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          r[j] = (active && x == 0) ? (uint32_t(__ldg(qr + 2 * j)) | (uint32_t(__ldg(qr + 2 * j + 1)) << 16))
-                                    : 0u;
-        tmem_st32(row_t + kColQr, r);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(QREADY);
+        tmem_st32(row_t + kColQ + 32 * half, r);
       }
+      const uint4* qr = qr_row(pc);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint4 u = (active && x == 0) ? __ldg(qr + j) : make_uint4(0u, 0u, 0u, 0u);
+        r[4 * j] = u.x; r[4 * j + 1] = u.y; r[4 * j + 2] = u.z; r[4 * j + 3] = u.w;
+      }
+      tmem_st32(row_t + kColQr, r);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(QREADY);
+    };
+    // pull the next piece's query rows into L2 while this piece streams
+    auto prefetch_q = [&](const Piece& pc) {
+      if (!active) return;
+      const char* q = reinterpret_cast<const char*>(q_row(pc));
+      prefetch_l2_evict_last(q + 256 * x);
+      prefetch_l2_evict_last(q + 256 * x + 128);
+      if (x == 0) prefetch_l2_evict_last(qr_row(pc));
+    };
+    Piece p, pn;
+    int it = 0;
+    bool ok = walk.next(p);
+    bool has_next = ok && walk.next(pn);
+    if (ok) write_q(p);
+    if (has_next) prefetch_q(pn);
+    while (ok) {
       float m = -INFINITY, l = 0.f;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int sb = it & 1;
@@ -372,26 +416,41 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) { v[k] = r0[k]; v[32 + k] = r1[k]; }
         }
+        // every QK of this piece is done: the next piece's queries can go in now
+        if (t + 1 == p.t1 && has_next) write_q(pn);
         const int valid = min(kTile, p.L - t * kTile);
-        float s[32];
-        float mt = -INFINITY;
+        float raw[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           const float send = __uint_as_float(x ? v[k] : v[32 + k]);
           const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-          const float own = __uint_as_float(x ? v[32 + k] : v[k]);
-          const int tok = 32 * x + k;
-          s[k] = (tok < valid) ? (own + recv) * sl2 : -INFINITY;
-          mt = fmaxf(mt, s[k]);
+          raw[k] = __uint_as_float(x ? v[32 + k] : v[k]) + recv;
         }
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+        if (valid < kTile) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (32 * x + k >= valid) raw[k] = -INFINITY;
+        }
+        float mx;
+        {
+          float t16[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) t16[k] = fmaxf(raw[k], raw[k + 16]);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) t16[k] = fmaxf(t16[k], t16[k + 8]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) t16[k] = fmaxf(t16[k], t16[k + 4]);
+          mx = fmaxf(fmaxf(t16[0], t16[2]), fmaxf(t16[1], t16[3]));
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float mt = mx * sl2;  // tile max in log2 units
         if (t == p.t0) {
           m = mt;
         } else if (mt > m + kRescaleLog2) {
-          const float alpha = exp2f(m - mt);
+          const float alpha = ex2_approx(m - mt);
           m = mt;
           l *= alpha;
-          // O must not be in use by the previous PV while it is rescaled
+          // this row of O must not be in use by the previous PV while it is rescaled
           const int pk = it - 1;
           if (!wait_bar(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
@@ -406,11 +465,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
           tmem_wait_st();
         }
+        const float neg_m = -m;
         float ls = 0.f;
         uint32_t whi[16], wlo[16];
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
-          const float p0 = exp2f(s[k] - m), p1 = exp2f(s[k + 1] - m);
+          const float p0 = ex2_approx(fmaf(raw[k], sl2, neg_m));
+          const float p1 = ex2_approx(fmaf(raw[k + 1], sl2, neg_m));
           ls += p0 + p1;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           const float2 hf = __bfloat1622float2(h2);
@@ -418,6 +479,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           wlo[k / 2] = pack_bf16(p0 - hf.x, p1 - hf.y);
         }
         l += ls;
+        // row hi (x=0) takes P_hi of all 64 tokens, row lo (x=1) P_lo; written over S
         uint32_t prow[32];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -463,7 +525,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (active && x == 0)
         lse_part[(size_t(p.slot) * H + head) * nb + branch] =
             l_tot > 0.f ? (m + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
-      ++piece;
+      if (!has_next) break;
+      p = pn;
+      has_next = walk.next(pn);
+      if (has_next) prefetch_q(pn);
     }
   }
 
@@ -488,8 +553,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Heads per CTA (a head group) and branches per CTA: the 128 MMA rows hold
+// G branches x HPC heads x (hi, lo).
+int hpc_of(const mlra_config_t& c) { return c.n_heads < 64 ? c.n_heads : 64; }
 int g_of(const mlra_config_t& c) {
-  const int per = 64 / c.n_heads;
+  const int per = 64 / hpc_of(c);
   return c.n_blocks < per ? c.n_blocks : per;
 }
 
@@ -513,13 +581,13 @@ cudaError_t launch_t(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t s
 
 bool tc_supported(const mlra_config_t& c) {
   if (c.dtype != MLRA_BF16 || c.d_cb != 128 || c.d_r != 64) return false;
-  if (c.n_heads != 16 && c.n_heads != 32 && c.n_heads != 64) return false;
+  if (c.n_heads != 16 && c.n_heads != 32 && c.n_heads != 64 && c.n_heads != 128) return false;
   if (c.n_blocks != 1 && c.n_blocks != 2 && c.n_blocks != 4) return false;
   return c.n_blocks % g_of(c) == 0;
 }
 
 void tc_grid(const mlra_config_t& c, int num_sms, int* n_groups, int* ctas_per_group) {
-  *n_groups = c.n_blocks / g_of(c);
+  *n_groups = (c.n_blocks / g_of(c)) * (c.n_heads / hpc_of(c));
   *ctas_per_group = num_sms / *n_groups > 0 ? num_sms / *n_groups : 1;
 }
 
@@ -540,8 +608,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  const int G = g_of(c);
-  switch (c.n_heads * 10 + G) {
+  switch (hpc_of(c) * 10 + g_of(c)) {
     case 164: return launch_t<4, 16>(map, a, st);
     case 162: return launch_t<2, 16>(map, a, st);
     case 161: return launch_t<1, 16>(map, a, st);

@@ -106,67 +106,111 @@ cudaError_t launch_plan(const int32_t* seqlens, int batch, int cap, int ctas_per
 
 // ---------------------------------------------------------------------------
 // Absorption: q_abs[s,h,b,i] = sum_j W_uk[b,h,i,j] q_nope[s,h,j]
-// Block (head h, 8 sequences); warp w takes latent rows (b,i) = w, w+8, ...;
-// lanes split j and reduce with shuffles.  W_uk is streamed once per block.
+// Block = (head h, 256 latent rows, 8 sequences), one thread per latent row
+// (b,i).  The thread issues every 16-byte load of its W_uk row (d_h contiguous
+// values) for a 64-wide chunk at once, then multiplies with q_nope of the 8
+// sequences read from shared memory as float4 (one address per warp:
+// broadcast).
 // ---------------------------------------------------------------------------
 constexpr int kSeqBlk = 8;
+constexpr int kAbsThreads = 256;
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&w)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __bfloat1622float2(h[k]);
+    w[2 * k] = f.x;
+    w[2 * k + 1] = f.y;
+  }
+}
+
+template <typename T> struct Chunk8;
+template <> struct Chunk8<__nv_bfloat16> {  // 8 bf16 = one 16-byte load
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void get(float (&w)[8]) const { unpack8(u, w); }
+};
+template <> struct Chunk8<float> {  // 8 fp32 = two 16-byte loads
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p + 4));
+  }
+  __device__ __forceinline__ void get(float (&w)[8]) const {
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+};
 
 template <typename T>
-__global__ void __launch_bounds__(256) absorb_kernel(const T* __restrict__ q_nope,
-                                                     const T* __restrict__ w_uk,
-                                                     float* __restrict__ q_abs, int batch,
-                                                     int heads, int nb, int d_cb, int d_h) {
-  extern __shared__ float sq[];  // [kSeqBlk][d_h]
-  const int h = blockIdx.x, s0 = blockIdx.y * kSeqBlk;
+__global__ void __launch_bounds__(kAbsThreads) absorb_kernel(const T* __restrict__ q_nope,
+                                                             const T* __restrict__ w_uk,
+                                                             float* __restrict__ q_abs, int batch,
+                                                             int heads, int nb, int d_cb, int d_h) {
+  extern __shared__ float4 sq4[];  // [kSeqBlk][d_h / 4]
+  float* sq = reinterpret_cast<float*>(sq4);
+  const int h = blockIdx.x, s0 = blockIdx.z * kSeqBlk;
   const int ns = min(kSeqBlk, batch - s0);
   for (int x = threadIdx.x; x < kSeqBlk * d_h; x += blockDim.x) {
-    int s = x / d_h, j = x % d_h;
+    const int s = x / d_h, j = x - s * d_h;
     sq[x] = (s < ns) ? ld_f32(q_nope + (size_t(s0 + s) * heads + h) * d_h + j) : 0.f;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int rows = nb * d_cb;
-  for (int r = warp; r < rows; r += 8) {
-    const int b = r / d_cb, i = r % d_cb;
-    const T* wrow = w_uk + ((size_t(b) * heads + h) * d_cb + i) * d_h;
-    float acc[kSeqBlk];
+  const int K = nb * d_cb;
+  const int r = blockIdx.y * kAbsThreads + threadIdx.x;
+  if (r >= K) return;
+  const int b = r / d_cb, i = r - b * d_cb;
+  const T* wrow = w_uk + ((size_t(b) * heads + h) * d_cb + i) * d_h;
+  float acc[kSeqBlk];
 #pragma unroll
-    for (int s = 0; s < kSeqBlk; ++s) acc[s] = 0.f;
-    for (int j = lane; j < d_h; j += 32) {
-      float w = ld_f32(wrow + j);
+  for (int s = 0; s < kSeqBlk; ++s) acc[s] = 0.f;
+  const int q4 = d_h / 4;
+  for (int j0 = 0; j0 < d_h; j0 += 64) {
+    const int nc = min(8, (d_h - j0) / 8);
+    Chunk8<T> c[8];
 #pragma unroll
-      for (int s = 0; s < kSeqBlk; ++s) acc[s] = fmaf(w, sq[s * d_h + j], acc[s]);
-    }
+    for (int k = 0; k < 8; ++k)
+      if (k < nc) c[k].load(wrow + j0 + 8 * k);
 #pragma unroll
-    for (int s = 0; s < kSeqBlk; ++s) {
+    for (int k = 0; k < 8; ++k) {
+      if (k >= nc) break;
+      float w[8];
+      c[k].get(w);
+      const int jq = (j0 + 8 * k) / 4;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[s] += __shfl_xor_sync(0xffffffffu, acc[s], o);
-    }
-    if (lane < ns) {
-      float v = acc[0];
-#pragma unroll
-      for (int s = 1; s < kSeqBlk; ++s) if (lane == s) v = acc[s];
-      q_abs[((size_t(s0 + lane) * heads + h) * nb + b) * d_cb + i] = v;
+      for (int s = 0; s < kSeqBlk; ++s) {
+        const float4 qa = sq4[s * q4 + jq], qb = sq4[s * q4 + jq + 1];
+        acc[s] = fmaf(w[0], qa.x, acc[s]); acc[s] = fmaf(w[1], qa.y, acc[s]);
+        acc[s] = fmaf(w[2], qa.z, acc[s]); acc[s] = fmaf(w[3], qa.w, acc[s]);
+        acc[s] = fmaf(w[4], qb.x, acc[s]); acc[s] = fmaf(w[5], qb.y, acc[s]);
+        acc[s] = fmaf(w[6], qb.z, acc[s]); acc[s] = fmaf(w[7], qb.w, acc[s]);
+      }
     }
   }
+  for (int s = 0; s < ns; ++s) q_abs[(size_t(s0 + s) * heads + h) * K + r] = acc[s];
 }
 
 cudaError_t launch_absorb(const mlra_config_t& c, const void* q_nope, const void* w_uk,
                           float* q_abs, int batch, cudaStream_t st) {
-  dim3 grid(c.n_heads, (batch + kSeqBlk - 1) / kSeqBlk);
+  dim3 grid(c.n_heads, (c.n_blocks * c.d_cb + kAbsThreads - 1) / kAbsThreads,
+            (batch + kSeqBlk - 1) / kSeqBlk);
   size_t sm = sizeof(float) * kSeqBlk * c.d_h;
   if (c.dtype == MLRA_BF16)
-    absorb_kernel<__nv_bfloat16><<<grid, 256, sm, st>>>(
+    absorb_kernel<__nv_bfloat16><<<grid, kAbsThreads, sm, st>>>(
         (const __nv_bfloat16*)q_nope, (const __nv_bfloat16*)w_uk, q_abs, batch, c.n_heads,
         c.n_blocks, c.d_cb, c.d_h);
   else
-    absorb_kernel<float><<<grid, 256, sm, st>>>((const float*)q_nope, (const float*)w_uk, q_abs,
-                                                batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h);
+    absorb_kernel<float><<<grid, kAbsThreads, sm, st>>>((const float*)q_nope, (const float*)w_uk,
+                                                        q_abs, batch, c.n_heads, c.n_blocks,
+                                                        c.d_cb, c.d_h);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Split-KV combine: one warp per (sequence, head, branch).
+// Split-KV combine: one warp per (sequence, head, branch).  Lane k reads the
+// lse of split k (32 splits per round), the merge weights come from warp
+// reductions, and each lane accumulates 4 consecutive latent values per split
+// with 16-byte loads (d_cb a multiple of 128 uses the vector path).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) combine_kernel(const char* __restrict__ ws, WsLayout L,
                                                       int batch, int heads, int nb, int d_cb,
@@ -184,30 +228,50 @@ __global__ void __launch_bounds__(256) combine_kernel(const char* __restrict__ w
   const size_t row = (size_t(h) * nb + b);
   const size_t slot_stride = size_t(heads) * nb;
   float* dst = o_latent + ((size_t(s) * heads + h) * nb + b) * d_cb;
-  if (k1 <= k0) {
-    for (int i = lane; i < d_cb; i += 32) dst[i] = 0.f;
-    if (lse_out && lane == 0) lse_out[(size_t(s) * heads + h) * nb + b] = -INFINITY;
-    return;
-  }
+  float* lse_dst = lse_out ? lse_out + (size_t(s) * heads + h) * nb + b : nullptr;
+  // max and sum of exp over the splits
   float m = -INFINITY;
-  for (int k = k0; k < k1; ++k) m = fmaxf(m, __ldg(lse_part + size_t(k) * slot_stride + row));
-  if (m == -INFINITY) {  // every token of the sequence was rejected (bad page)
+  for (int k = k0 + lane; k < k1; k += 32) m = fmaxf(m, __ldg(lse_part + size_t(k) * slot_stride + row));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (k1 <= k0 || m == -INFINITY) {  // no token (empty sequence / every page rejected)
     for (int i = lane; i < d_cb; i += 32) dst[i] = 0.f;
-    if (lse_out && lane == 0) lse_out[(size_t(s) * heads + h) * nb + b] = -INFINITY;
+    if (lse_dst && lane == 0) *lse_dst = -INFINITY;
     return;
   }
   float den = 0.f;
-  for (int k = k0; k < k1; ++k) den += expf(__ldg(lse_part + size_t(k) * slot_stride + row) - m);
+  for (int k = k0 + lane; k < k1; k += 32) den += expf(__ldg(lse_part + size_t(k) * slot_stride + row) - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   const float inv = 1.f / den;
-  for (int i = lane; i < d_cb; i += 32) {
-    float acc = 0.f;
-    for (int k = k0; k < k1; ++k) {
-      float w = expf(__ldg(lse_part + size_t(k) * slot_stride + row) - m);
-      acc = fmaf(w, __ldg(o_part + (size_t(k) * slot_stride + row) * d_cb + i), acc);
+  if ((d_cb & 127) == 0) {
+    for (int i0 = 0; i0 < d_cb; i0 += 128) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int kb = k0; kb < k1; kb += 32) {
+        const int k = kb + lane;
+        const float wl = (k < k1) ? expf(__ldg(lse_part + size_t(k) * slot_stride + row) - m) * inv : 0.f;
+        const int nk = min(32, k1 - kb);
+        for (int j = 0; j < nk; ++j) {
+          const float w = __shfl_sync(0xffffffffu, wl, j);
+          const float4 o = __ldg(reinterpret_cast<const float4*>(
+              o_part + (size_t(kb + j) * slot_stride + row) * d_cb + i0 + 4 * lane));
+          acc.x = fmaf(w, o.x, acc.x); acc.y = fmaf(w, o.y, acc.y);
+          acc.z = fmaf(w, o.z, acc.z); acc.w = fmaf(w, o.w, acc.w);
+        }
+      }
+      *reinterpret_cast<float4*>(dst + i0 + 4 * lane) = acc;
     }
-    dst[i] = acc * inv;
+  } else {
+    for (int i = lane; i < d_cb; i += 32) {
+      float acc = 0.f;
+      for (int k = k0; k < k1; ++k) {
+        const float w = expf(__ldg(lse_part + size_t(k) * slot_stride + row) - m) * inv;
+        acc = fmaf(w, __ldg(o_part + (size_t(k) * slot_stride + row) * d_cb + i), acc);
+      }
+      dst[i] = acc;
+    }
   }
-  if (lse_out && lane == 0) lse_out[(size_t(s) * heads + h) * nb + b] = m + logf(den);
+  if (lse_dst && lane == 0) *lse_dst = m + logf(den);
 }
 
 cudaError_t launch_combine(const mlra_config_t& c, const void* ws, const WsLayout& L, int batch,
@@ -222,68 +286,117 @@ cudaError_t launch_combine(const mlra_config_t& c, const void* ws, const WsLayou
 
 // ---------------------------------------------------------------------------
 // Output up-projection: out[s,h,j] = branch_scale * sum_{b,i} o[s,h,b,i] W_uv[b,h,i,j]
-// Block (head h, 8 sequences); W_uv rows are staged through shared memory in
-// chunks of 32 latent rows; warp w owns sequence s0+w, lanes own columns j.
+// Block = (head h, 8 sequences), 8 warps.  Warp w sums the latent rows k=(b,i)
+// of its eighth of K = nb*d_cb; lane l owns output columns 4l..4l+3 (one
+// coalesced row segment of W_uv per warp and k, read as 4 values per lane).
+// o of the 8 sequences is kept transposed in shared memory ([k][s], two
+// float4 per k, broadcast across the warp); the eight warps' partial sums are
+// added through shared memory.
 // ---------------------------------------------------------------------------
-constexpr int kKChunk = 32;
+constexpr int kOpWarps = 8;
+
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float4 load4(const float* p) {
+  return __ldg(reinterpret_cast<const float4*>(p));
+}
 
 template <typename T>
-__global__ void __launch_bounds__(256) out_proj_kernel(const float* __restrict__ o_lat,
-                                                       const T* __restrict__ w_uv,
-                                                       float* __restrict__ out, int batch,
-                                                       int heads, int nb, int d_cb, int d_h,
-                                                       float branch_scale) {
-  extern __shared__ float sm[];
-  float* sw = sm;                       // [kKChunk][d_h]
-  float* so = sm + kKChunk * d_h;       // [kSeqBlk][kKChunk]
+__global__ void __launch_bounds__(kOpWarps * 32) out_proj_kernel(const float* __restrict__ o_lat,
+                                                                 const T* __restrict__ w_uv,
+                                                                 float* __restrict__ out, int batch,
+                                                                 int heads, int nb, int d_cb,
+                                                                 int d_h, float branch_scale) {
+  extern __shared__ float4 sm4[];
+  const int K = nb * d_cb;
+  float* so = reinterpret_cast<float*>(sm4);    // [K][kSeqBlk]
+  float* red = so + size_t(K) * kSeqBlk;        // [kOpWarps][kSeqBlk][d_h]
   const int h = blockIdx.x, s0 = blockIdx.y * kSeqBlk;
   const int ns = min(kSeqBlk, batch - s0);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int K = nb * d_cb;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // columns lane + 32 q, q < d_h / 32 (d_h <= 128)
-  for (int k0 = 0; k0 < K; k0 += kKChunk) {
-    __syncthreads();
-    for (int x = threadIdx.x; x < kKChunk * d_h; x += blockDim.x) {
-      int kk = x / d_h, j = x % d_h, k = k0 + kk;
-      int b = k / d_cb, i = k % d_cb;
-      sw[x] = ld_f32(w_uv + ((size_t(b) * heads + h) * d_cb + i) * d_h + j);
-    }
-    for (int x = threadIdx.x; x < kSeqBlk * kKChunk; x += blockDim.x) {
-      int s = x / kKChunk, kk = x % kKChunk, k = k0 + kk;
-      so[x] = (s < ns) ? __ldg(o_lat + (size_t(s0 + s) * heads + h) * K + k) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kKChunk; ++kk) {
-      const float o = so[warp * kKChunk + kk];
+  for (int x = threadIdx.x; x < kSeqBlk * K; x += blockDim.x) {
+    const int s = x / K, k = x - s * K;
+    so[k * kSeqBlk + s] = (s < ns) ? __ldg(o_lat + (size_t(s0 + s) * heads + h) * K + k) : 0.f;
+  }
+  __syncthreads();
+  const int c0 = 4 * lane;
+  const bool cok = c0 < d_h;
+  float4 acc[kSeqBlk];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        int j = lane + 32 * q;
-        if (j < d_h) acc[q] = fmaf(o, sw[kk * d_h + j], acc[q]);
+  for (int s = 0; s < kSeqBlk; ++s) acc[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int per = K / kOpWarps;  // K is a multiple of 8
+  const int k0 = warp * per, k1 = k0 + per;
+  int b = k0 / d_cb, i = k0 - b * d_cb;
+  const T* wp = w_uv + ((size_t(b) * heads + h) * d_cb + i) * d_h + c0;
+  for (int k = k0; k < k1; k += 8) {
+    float4 w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {  // 8 rows in flight
+      w[u] = cok ? load4(wp) : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (++i == d_cb) { i = 0; ++b; wp = w_uv + (size_t(b) * heads + h) * d_cb * d_h + c0; }
+      else wp += d_h;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 oa = *reinterpret_cast<const float4*>(so + (k + u) * kSeqBlk);
+      const float4 ob = *reinterpret_cast<const float4*>(so + (k + u) * kSeqBlk + 4);
+      const float o[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
+#pragma unroll
+      for (int s = 0; s < kSeqBlk; ++s) {
+        acc[s].x = fmaf(o[s], w[u].x, acc[s].x); acc[s].y = fmaf(o[s], w[u].y, acc[s].y);
+        acc[s].z = fmaf(o[s], w[u].z, acc[s].z); acc[s].w = fmaf(o[s], w[u].w, acc[s].w);
       }
     }
   }
-  if (warp < ns) {
+  if (cok) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      int j = lane + 32 * q;
-      if (j < d_h) out[(size_t(s0 + warp) * heads + h) * d_h + j] = branch_scale * acc[q];
-    }
+    for (int s = 0; s < kSeqBlk; ++s)
+      *reinterpret_cast<float4*>(red + (size_t(warp) * kSeqBlk + s) * d_h + c0) = acc[s];
+  }
+  __syncthreads();
+  for (int x = threadIdx.x; x < kSeqBlk * d_h; x += blockDim.x) {
+    const int s = x / d_h, j = x - s * d_h;
+    if (s >= ns) continue;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kOpWarps; ++w) v += red[(size_t(w) * kSeqBlk + s) * d_h + j];
+    out[(size_t(s0 + s) * heads + h) * d_h + j] = branch_scale * v;
   }
 }
 
 cudaError_t launch_out_proj(const mlra_config_t& c, const float* o_latent, const void* w_uv,
                             float* out, int batch, cudaStream_t st) {
+  if ((c.n_blocks * c.d_cb) % 64 != 0 || c.d_h % 4 != 0) return cudaErrorInvalidValue;
   dim3 grid(c.n_heads, (batch + kSeqBlk - 1) / kSeqBlk);
-  size_t sm = sizeof(float) * (kKChunk * c.d_h + kSeqBlk * kKChunk);
+  const size_t sm = sizeof(float) * (size_t(c.n_blocks) * c.d_cb * kSeqBlk +
+                                     size_t(kOpWarps) * kSeqBlk * c.d_h);
+  if (sm > 48 * 1024) {
+    // opt in once per device to the shared memory a wide latent needs
+    static int set_for[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || set_for[dev] < (int)sm) {
+      cudaError_t e = cudaFuncSetAttribute(out_proj_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(out_proj_kernel<float>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) set_for[dev] = (int)sm;
+    }
+  }
   if (c.dtype == MLRA_BF16)
-    out_proj_kernel<__nv_bfloat16><<<grid, 256, sm, st>>>(
+    out_proj_kernel<__nv_bfloat16><<<grid, kOpWarps * 32, sm, st>>>(
         o_latent, (const __nv_bfloat16*)w_uv, out, batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h,
         c.branch_scale);
   else
-    out_proj_kernel<float><<<grid, 256, sm, st>>>(o_latent, (const float*)w_uv, out, batch,
-                                                  c.n_heads, c.n_blocks, c.d_cb, c.d_h,
-                                                  c.branch_scale);
+    out_proj_kernel<float><<<grid, kOpWarps * 32, sm, st>>>(o_latent, (const float*)w_uv, out,
+                                                            batch, c.n_heads, c.n_blocks, c.d_cb,
+                                                            c.d_h, c.branch_scale);
   return cudaGetLastError();
 }
 

@@ -120,6 +120,8 @@ mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const 
   if (batch < 0) return MLRA_ERR_INVALID_ARG;
   if (batch == 0) return MLRA_OK;
   if (!q_nope || !w_uk || !q_abs) return MLRA_ERR_INVALID_ARG;
+  if (!aligned(w_uk, 16) || !aligned(q_nope, cfg->dtype == MLRA_BF16 ? 2 : 4) || !aligned(q_abs, 4))
+    return MLRA_ERR_ALIGNMENT;
   return from_cuda(launch_absorb(*cfg, q_nope, w_uk, q_abs, batch, (cudaStream_t)stream));
 }
 
@@ -150,8 +152,7 @@ mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, con
     if (cfg->page_size != kPageSize) return MLRA_ERR_UNSUPPORTED;
     if (num_pages < 1 || num_pages > (int64_t(1) << 31) / kPageSize) return MLRA_ERR_INVALID_ARG;
   }
-  const uintptr_t elt = cfg->dtype == MLRA_BF16 ? 2 : 4;
-  if (!aligned(kv_cache, 16) || !aligned(q_abs, 4) || !aligned(q_rope, elt) ||
+  if (!aligned(kv_cache, 16) || !aligned(q_abs, 16) || !aligned(q_rope, 16) ||
       !aligned(seqlens, 4) || (page_table && !aligned(page_table, 4)))
     return MLRA_ERR_ALIGNMENT;
   Grid g;
@@ -208,6 +209,7 @@ mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, con
   if (batch < 0) return MLRA_ERR_INVALID_ARG;
   if (batch == 0) return MLRA_OK;
   if (!o_latent || !w_uv || !out) return MLRA_ERR_INVALID_ARG;
+  if (!aligned(w_uv, 16) || !aligned(o_latent, 4) || !aligned(out, 4)) return MLRA_ERR_ALIGNMENT;
   return from_cuda(launch_out_proj(*cfg, o_latent, w_uv, out, batch, (cudaStream_t)stream));
 }
 

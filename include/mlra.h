@@ -99,7 +99,7 @@ MLRA_API int32_t mlra_version(void);
  *   q_nope : [batch, n_heads, d_h]            dtype
  *   w_uk   : [n_blocks, n_heads, d_cb, d_h]   dtype
  *   q_abs  : [batch, n_heads, n_blocks, d_cb] fp32 (written)
- * fp32 accumulation.  batch = 0 is a no-op.
+ * fp32 accumulation.  batch = 0 is a no-op.  w_uk must be 16-byte aligned.
  */
 MLRA_API mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const void* w_uk,
                             float* q_abs, int32_t batch, mlra_stream_t stream);
@@ -136,9 +136,9 @@ MLRA_API mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t bat
  *   workspace  : >= mlra_workspace_size bytes, 256-byte aligned, caller-owned
  * Cache rows at or beyond seqlens[s] never influence the result, whatever they
  * hold (they are zero-filled on chip before use).  The device error word is
- * reset at the start of every call.  kv_cache must be 16-byte aligned (it is
- * read by the tensor-memory accelerator); the other pointers need only the
- * alignment of their element type.
+ * reset at the start of every call.  kv_cache, q_abs and q_rope must be
+ * 16-byte aligned (they are read in 16-byte units, the cache by the tensor
+ * memory accelerator); seqlens and page_table 4-byte aligned.
  */
 MLRA_API mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, const void* q_rope,
                                const void* kv_cache, int64_t num_pages, const int32_t* page_table,
@@ -164,6 +164,7 @@ MLRA_API mlra_status_t mlra_splitkv_combine(const mlra_config_t* cfg, const void
  *   o_latent : [batch, n_heads, n_blocks, d_cb] fp32
  *   w_uv     : [n_blocks, n_heads, d_cb, d_h] dtype
  *   out      : [batch, n_heads, d_h] fp32 (written)
+ * w_uv must be 16-byte aligned; d_h <= 128.
  */
 MLRA_API mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, const void* w_uv,
                             float* out, int32_t batch, mlra_stream_t stream);
