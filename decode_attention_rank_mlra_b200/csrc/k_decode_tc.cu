@@ -42,9 +42,6 @@ constexpr uint32_t kColQ = 0;                // q_abs rows (bf16 pairs): 64 colu
 constexpr uint32_t kColQr = 64;              // q_rope rows: 32 columns
 constexpr uint32_t kColS = 128;              // S / P double buffer: 2 x 64 columns
 constexpr uint32_t kColO = 256;              // O accumulator: 128 columns
-// A row keeps its running max until a tile exceeds it by 2^8; the O rescale that
-// follows is done by the row's own thread on its own TMEM lane.
-constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kSmemLimit = 232448;           // max dynamic shared memory per block
 
@@ -334,13 +331,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warps 0-3
-    // Thread = one row (TMEM lane): branch bg, head, hi (x=0) or lo (x=1) part.
-    // The hi and lo rows of a head sit 16 lanes apart and trade halves with
-    // shuffles; every other step is the thread's own.
+    // Thread = one TMEM lane of the quadrant: branch bg, head, and x = lane / 16,
+    // which is the row the thread writes the queries of (0: hi, 1: lo) and the
+    // half of each tile's 64 tokens it takes the softmax of.
     const int bg = warp / WPB;
     const int branch = g * G + bg;
     const bool active = bg < G && branch < nb;
-    const int x = lane >> 4;                                 // 0: hi row, 1: lo row
+    const int x = lane >> 4;
     const int head = head0 + 16 * (warp % WPB) + (lane & 15);
     const uint32_t row_t = tmem + (uint32_t(32 * warp) << 16);
     const float sl2 = a.cfg.softmax_scale * 1.4426950408889634f;
@@ -395,6 +392,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       prefetch_l2_evict_last(q + 256 * x + 128);
       if (x == 0) prefetch_l2_evict_last(qr_row(pc));
     };
+    // Lanes 0-15 of the quadrant hold the hi rows and lanes 16-31 the lo rows of
+    // the same 16 heads.  The .16x32bx2 TMEM accesses give thread t (< 16) both
+    // rows of head t for tokens 0-31 and thread t + 16 both rows for tokens
+    // 32-63, so S_hi + S_lo, the P_hi / P_lo write-back and O_hi + O_lo need no
+    // shuffles.
+    const uint32_t hi_t = row_t;                   // lane base 0 of the quadrant
+    const uint32_t lo_t = row_t + (16u << 16);     // lane base 16
     Piece p, pn;
     int it = 0;
     bool ok = walk.next(p);
@@ -402,37 +406,32 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if (ok) write_q(p);
     if (has_next) prefetch_q(pn);
     while (ok) {
+      // m: the reference point of the exponentials, in log2 units.  It is the
+      // first tile's max and moves only when a later tile would overflow
+      // (2^64 above it); a stale m only shifts all weights by the same factor.
       float m = -INFINITY, l = 0.f;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int sb = it & 1;
         if (!wait_bar(SFULL(sb), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        uint32_t v[64];
+        float raw[32];
         {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(row_t + kColS + 64 * sb, r0);
-          tmem_ld32(row_t + kColS + 64 * sb + 32, r1);
+          uint32_t sh[32], sl[32];
+          tmem_ld_x2_32<32>(hi_t + kColS + 64 * sb, sh);
+          tmem_ld_x2_32<32>(lo_t + kColS + 64 * sb, sl);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) { v[k] = r0[k]; v[32 + k] = r1[k]; }
+          for (int k = 0; k < 32; ++k) raw[k] = __uint_as_float(sh[k]) + __uint_as_float(sl[k]);
         }
         // every QK of this piece is done: the next piece's queries can go in now
         if (t + 1 == p.t1 && has_next) write_q(pn);
         const int valid = min(kTile, p.L - t * kTile);
-        float raw[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float send = __uint_as_float(x ? v[k] : v[32 + k]);
-          const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-          raw[k] = __uint_as_float(x ? v[32 + k] : v[k]) + recv;
-        }
         if (valid < kTile) {
 #pragma unroll
           for (int k = 0; k < 32; ++k)
             if (32 * x + k >= valid) raw[k] = -INFINITY;
         }
-        float mx;
-        {
+        auto tile_max = [&]() {
           float t16[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) t16[k] = fmaxf(raw[k], raw[k + 16]);
@@ -440,54 +439,55 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           for (int k = 0; k < 8; ++k) t16[k] = fmaxf(t16[k], t16[k + 8]);
 #pragma unroll
           for (int k = 0; k < 4; ++k) t16[k] = fmaxf(t16[k], t16[k + 4]);
-          mx = fmaxf(fmaxf(t16[0], t16[2]), fmaxf(t16[1], t16[3]));
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float mt = mx * sl2;  // tile max in log2 units
-        if (t == p.t0) {
-          m = mt;
-        } else if (mt > m + kRescaleLog2) {
-          const float alpha = ex2_approx(m - mt);
-          m = mt;
-          l *= alpha;
-          // this row of O must not be in use by the previous PV while it is rescaled
-          const int pk = it - 1;
-          if (!wait_bar(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(row_t + kColO + 32 * ch, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            tmem_st32(row_t + kColO + 32 * ch, r);
-          }
-          tmem_wait_st();
-        }
-        const float neg_m = -m;
-        float ls = 0.f;
+          const float mx = fmaxf(fmaxf(t16[0], t16[2]), fmaxf(t16[1], t16[3]));
+          return fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * sl2;
+        };
+        if (t == p.t0) m = tile_max();
         uint32_t whi[16], wlo[16];
+        float ls;
+        auto exps = [&]() {
+          const float neg_m = -m;
+          ls = 0.f;
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const float p0 = ex2_approx(fmaf(raw[k], sl2, neg_m));
-          const float p1 = ex2_approx(fmaf(raw[k + 1], sl2, neg_m));
-          ls += p0 + p1;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          const float2 hf = __bfloat1622float2(h2);
-          whi[k / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-          wlo[k / 2] = pack_bf16(p0 - hf.x, p1 - hf.y);
+          for (int k = 0; k < 32; k += 2) {
+            const float p0 = ex2_approx(fmaf(raw[k], sl2, neg_m));
+            const float p1 = ex2_approx(fmaf(raw[k + 1], sl2, neg_m));
+            ls += p0 + p1;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            const float2 hf = __bfloat1622float2(h2);
+            whi[k / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+            wlo[k / 2] = pack_bf16(p0 - hf.x, p1 - hf.y);
+          }
+        };
+        exps();
+        if (__any_sync(0xffffffffu, !(ls <= 0x1p64f))) {
+          // rare: a score far above m (or a NaN).  Raise m to this tile's max,
+          // rescale l and the O rows once the previous PV is done, redo the tile.
+          const float mt = tile_max();
+          if (mt > m) {
+            const float alpha = ex2_approx(m - mt);
+            m = mt;
+            l *= alpha;
+            const int pk = it - 1;
+            if (!wait_bar(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t r[32];
+              tmem_ld32(row_t + kColO + 32 * ch, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+              tmem_st32(row_t + kColO + 32 * ch, r);
+            }
+            tmem_wait_st();
+          }
+          exps();
         }
         l += ls;
-        // row hi (x=0) takes P_hi of all 64 tokens, row lo (x=1) P_lo; written over S
-        uint32_t prow[32];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t recv = __shfl_xor_sync(0xffffffffu, x ? whi[j] : wlo[j], 16);
-          prow[j] = x ? recv : whi[j];
-          prow[16 + j] = x ? wlo[j] : recv;
-        }
-        tmem_st32(row_t + kColS + 64 * sb, prow);
+        // P over S: the hi row of head t takes P_hi of all 64 tokens, the lo row P_lo
+        tmem_st_x2_16<16>(hi_t + kColS + 64 * sb, whi);
+        tmem_st_x2_16<16>(lo_t + kColS + 64 * sb, wlo);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -505,21 +505,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       float* dst = o_part + ((size_t(p.slot) * H + head) * nb + branch) * 128;
 #pragma unroll 1
       for (int j = 0; j < 2; ++j) {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(row_t + kColO + 32 * j, ra);
-        tmem_ld32(row_t + kColO + 64 + 32 * j, rb);
+        // thread t: features 32j.., thread t + 16: features 64 + 32j..
+        uint32_t oh[32], ol[32];
+        tmem_ld_x2_32<64>(hi_t + kColO + 32 * j, oh);
+        tmem_ld_x2_32<64>(lo_t + kColO + 32 * j, ol);
         tmem_wait_ld();
-        float o[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float send = __uint_as_float(x ? ra[k] : rb[k]);
-          const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-          o[k] = (__uint_as_float(x ? rb[k] : ra[k]) + recv) * inv;
-        }
         if (active) {
           float4* d4 = reinterpret_cast<float4*>(dst + 64 * x + 32 * j);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) d4[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+          for (int k = 0; k < 8; ++k)
+            d4[k] = make_float4((__uint_as_float(oh[4 * k]) + __uint_as_float(ol[4 * k])) * inv,
+                                (__uint_as_float(oh[4 * k + 1]) + __uint_as_float(ol[4 * k + 1])) * inv,
+                                (__uint_as_float(oh[4 * k + 2]) + __uint_as_float(ol[4 * k + 2])) * inv,
+                                (__uint_as_float(oh[4 * k + 3]) + __uint_as_float(ol[4 * k + 3])) * inv);
         }
       }
       if (active && x == 0)

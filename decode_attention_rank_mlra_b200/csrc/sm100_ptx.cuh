@@ -143,6 +143,27 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       MLRA_W8(0), MLRA_W8(8)
       : "memory");
 }
+// .16x32bx2 shapes: threads 0-15 access lanes base..base+15 at column c,
+// threads 16-31 the same lanes at column c + SPLIT.  With the lane base at 0
+// or 16 of the warp's quadrant this hands a row's columns to the partner half
+// of the warp without shuffles.
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld_x2_32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31}, [%32], %33;"
+      : MLRA_R8(0), MLRA_R8(8), MLRA_R8(16), MLRA_R8(24)
+      : "r"(taddr), "n"(SPLIT));
+}
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st_x2_16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, {%2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17};" ::"r"(taddr), "n"(SPLIT),
+      MLRA_W8(0), MLRA_W8(8)
+      : "memory");
+}
 #undef MLRA_R8
 #undef MLRA_W8
 

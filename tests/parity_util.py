@@ -74,5 +74,35 @@ def compare_batch(inp: W.DecodeInputs, got: Dict[str, torch.Tensor],
     finite = np.isfinite(lse_ref)
     assert np.array_equal(finite, np.isfinite(lse_got))
     if finite.any():
-        assert np.max(np.abs(lse_got[finite] - lse_ref[finite])) < (1e-5 if spec.dtype == "f32" else 2e-3)
+        d = np.abs(lse_got[finite] - lse_ref[finite])
+        if spec.dtype == "f32":
+            tol = 1e-5 * (1.0 + np.abs(lse_ref[finite]))
+        else:
+            # A logit reaches the softmax with an error of about 2^-15 of
+            # scale * sum_j |q_j k_j| (bf16 hi + lo queries, fp32 accumulation
+            # over 192 or 576 products), which can exceed |logit| many times
+            # over when the products cancel; the lse inherits it.
+            tol = 2e-3 + 2.0 ** -15 * logit_magnitude(inp, seqs, hs)[finite]
+        worst = int(np.argmax(d - tol))
+        assert np.all(d <= tol), f"lse err {d[worst]:.3e} > tol {tol[worst]:.3e}"
     return stats
+
+
+def logit_magnitude(inp: W.DecodeInputs, seqs: Sequence[int], heads: Sequence[int]) -> np.ndarray:
+    """[seq, head, branch] max over tokens of scale * sum_j |q_j k_j| (latent + RoPE)."""
+    from oracle.mlra_oracle import split_cache_rows
+    spec = inp.spec
+    nb = spec.n_blocks
+    out = np.zeros((len(seqs), len(heads), nb))
+    for i, s in enumerate(seqs):
+        rows = W.sequence_cache(inp, s)
+        if rows.shape[0] == 0:
+            continue
+        c, kr = split_cache_rows(rows.cpu(), nb, spec.d_cb)    # [L, nb, d_cb], [L, d_r]
+        qa = np.abs(oracle.absorb_query(inp.q_nope[s].cpu(), inp.w_uk.cpu()))  # [H, nb, d_cb]
+        qr = np.abs(inp.q_rope[s].cpu().double().numpy())      # [H, d_r]
+        rope = qr[heads] @ np.abs(kr).T                        # [h, L]
+        for b in range(nb):
+            lat = qa[heads, b] @ np.abs(c[:, b]).T             # [h, L]
+            out[i, :, b] = spec.softmax_scale * np.max(lat + rope, axis=1)
+    return out

@@ -95,6 +95,30 @@ def test_paged_tail_rows_never_matter():
         assert torch.equal(got[k], ref[k]), k
 
 
+def test_scores_rising_far_above_the_first_tile():
+    """Later tiles score hundreds of log2 units above the first tile's max: the
+    running reference point of the exponentials must move (no overflow)."""
+    inp = _small("mlra4_bf16_b16_h16_l4096_contig", 2, [700, 130])
+    inp.kv_cache[0, 64:700] *= 3000.0
+    inp.kv_cache[1, 100:130] *= 3000.0
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    compare_batch(inp, got)
+
+
+def test_scores_falling_far_below_the_first_tile():
+    """The first tile holds the largest scores by far: later weights underflow."""
+    inp = _small("mlra4_bf16_b64_h32_l16384_paged", 2, [300, 129])
+    flat = inp.kv_cache.view(-1, inp.spec.D)
+    pt = inp.page_table.cpu()
+    for s in range(2):
+        p0 = int(pt[s, 0]) * 64
+        flat[p0 + 3: p0 + 9] *= 3000.0
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    compare_batch(inp, got)
+
+
 def test_page_permutation_invariance():
     """Moving pages together with the page table leaves every output unchanged."""
     inp = _small("mlra4_bf16_b128_h16_ragged1k_64k_paged", 3, [300, 1000, 65])
