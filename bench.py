@@ -2,8 +2,9 @@
 """Benchmark of one MLRA / MLA latent-KV decode step on B200.
 
 A step is the whole hot path: absorb_q -> decode_attn (plan + split-KV
-attention) -> splitkv_combine -> out_proj, through the C ABI, on one batch of
-synthetic seeded inputs already resident in HBM.
+attention) -> combine_out_proj (split-KV merge fused with the output
+projection), through the C ABI, on one batch of synthetic seeded inputs
+already resident in HBM.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference] [--no-cpu-baseline]
@@ -215,8 +216,8 @@ def run_ours(args):
         mlra.absorb_q(cfg, q_nope, inp.w_uk, dec.q_abs)
         mlra.decode_attn(cfg, dec.q_abs, q_rope, caches[i % copies], inp.page_table, seqlens,
                          max_pages, dec.workspace)
-        mlra.splitkv_combine(cfg, dec.workspace, B, dec.o_latent, dec.lse)
-        return mlra.out_proj(cfg, dec.o_latent, inp.w_uv, dec.out)
+        return mlra.combine_out_proj(cfg, dec.workspace, B, inp.w_uv, dec.out, dec.o_latent,
+                                     dec.lse)
 
     for i in range(args.warmup):
         step(i)
@@ -275,40 +276,37 @@ def run_ours(args):
         kev[i][1].record(stream)
     torch.cuda.synchronize()
     k_ms = [a.elapsed_time(b) for a, b in kev]
-    # ---- per-call breakdown: each call captured alone in a CUDA graph and
-    # replayed back to back, one event pair around all replays -----------------
+    # ---- per-call breakdown: each call captured N times back to back in one
+    # CUDA graph (device time per call, no host launch gaps) -------------------
     calls = {
         "absorb_q": lambda i: mlra.absorb_q(cfg, inp.q_nope, inp.w_uk, dec.q_abs),
         "decode_attn": lambda i: mlra.decode_attn(cfg, dec.q_abs, inp.q_rope, caches[i % copies],
                                                   inp.page_table, inp.seqlens, max_pages,
                                                   dec.workspace),
-        "splitkv_combine": lambda i: mlra.splitkv_combine(cfg, dec.workspace, B, dec.o_latent,
-                                                          dec.lse),
-        "out_proj": lambda i: mlra.out_proj(cfg, dec.o_latent, inp.w_uv, dec.out),
+        "combine_out_proj": lambda i: mlra.combine_out_proj(cfg, dec.workspace, B, inp.w_uv,
+                                                            dec.out, dec.o_latent, dec.lse),
     }
     breakdown = {}
-    reps = max(10, min(args.steps, 200))
+    n_rep = 2 * copies
     for name, fn in calls.items():
-        gs = []
+        g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(side):
-            for i in range(copies):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=side):
+            with torch.cuda.graph(g, stream=side):
+                for i in range(n_rep):
                     fn(i)
-                gs.append(g)
         stream.wait_stream(side)
-        for i in range(2 * copies):
-            gs[i % copies].replay()
+        g.replay()
         torch.cuda.synchronize()
         b0 = torch.cuda.Event(enable_timing=True)
         b1 = torch.cuda.Event(enable_timing=True)
+        reps = max(3, min(50, args.steps // n_rep))
         b0.record(stream)
-        for i in range(reps):
-            gs[i % copies].replay()
+        for _ in range(reps):
+            g.replay()
         b1.record(stream)
         torch.cuda.synchronize()
-        breakdown[name] = b0.elapsed_time(b1) * 1e3 / reps
-        del gs
+        breakdown[name] = b0.elapsed_time(b1) * 1e3 / (reps * n_rep)
+        del g
     # ---- end-to-end: host buffers, copies inside the timed region ------------
     h_qn = inp.q_nope.cpu().pin_memory()
     h_qr = inp.q_rope.cpu().pin_memory()
@@ -383,8 +381,8 @@ def run_ours(args):
                             "the KV cache is device-resident state"},
             "clocks": clocks,
             "breakdown_us": breakdown,
-            "gpu_launches": 5 * args.steps,
-            "timing": "K replays of a CUDA graph of the whole step (5 kernels), one event pair around all K",
+            "gpu_launches": 4 * args.steps,
+            "timing": "K replays of a CUDA graph of the whole step (4 kernels), one event pair around all K",
         }
         if not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(spec, args.cpu_seconds)

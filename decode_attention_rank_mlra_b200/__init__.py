@@ -37,7 +37,7 @@ STATUS = {
 EXPORTS = [
     "mlra_status_string", "mlra_version", "mlra_absorb_q", "mlra_workspace_size",
     "mlra_decode_attn", "mlra_splitkv_combine", "mlra_out_proj", "mlra_get_device_error",
-    "mlra_decode_kernel_kind", "mlra_decode_attn_noalloc",
+    "mlra_decode_kernel_kind", "mlra_decode_attn_noalloc", "mlra_combine_out_proj",
 ]
 
 
@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
         "mlra_decode_attn": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, SZ, P]),
         "mlra_splitkv_combine": (I32, [CP, P, SZ, I32, P, P, P]),
         "mlra_out_proj": (I32, [CP, P, P, P, I32, P]),
+        "mlra_combine_out_proj": (I32, [CP, P, SZ, I32, P, P, P, P, P]),
         "mlra_get_device_error": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "mlra_decode_kernel_kind": (I32, [CP]),
         "mlra_decode_attn_noalloc": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, P, P, P]),
@@ -224,6 +225,29 @@ def out_proj(cfg: Config, o_latent: torch.Tensor, w_uv: torch.Tensor,
     return out
 
 
+def combine_out_proj(cfg: Config, workspace: torch.Tensor, batch: int, w_uv: torch.Tensor,
+                     out: Optional[torch.Tensor] = None, o_latent: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Steps 2b + 3 fused: merge the split partials and project (fp32 out).
+
+    ``o_latent`` / ``lse`` are written when given (needed when the fused
+    tensor-core kernel does not apply).
+    """
+    _need(w_uv, "w_uv", cfg.torch_dtype)
+    if out is None:
+        out = torch.empty((batch, cfg.n_heads, cfg.d_h), dtype=torch.float32,
+                          device=workspace.device)
+    _need(out, "out", torch.float32)
+    if o_latent is not None:
+        _need(o_latent, "o_latent", torch.float32)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    _check("mlra_combine_out_proj", lib().mlra_combine_out_proj(
+        ctypes.byref(cfg), _ptr(workspace), workspace.numel(), batch, _ptr(w_uv), _ptr(out),
+        _ptr(o_latent), _ptr(lse), _stream(stream)))
+    return out
+
+
 def decode_attn_noalloc(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor,
                         kv_cache: torch.Tensor, page_table: Optional[torch.Tensor],
                         seqlens: torch.Tensor, max_pages: int, o_latent: torch.Tensor,
@@ -277,7 +301,8 @@ class Decoder:
     """One layer's decode step with preallocated outputs and workspace.
 
     ``run`` launches absorb -> decode_attn -> splitkv_combine -> out_proj on
-    the current stream and returns ``out`` [B, h, d_h] fp32.
+    the current stream and returns ``out`` [B, h, d_h] fp32; with
+    ``fused=True`` the last two are one combine_out_proj call.
     """
 
     cfg: Config
@@ -294,18 +319,22 @@ class Decoder:
         self.out = torch.empty((B, c.n_heads, c.d_h), dtype=torch.float32, device=dev)
 
     def run(self, q_nope, q_rope, w_uk, w_uv, kv_cache, page_table, seqlens, max_pages,
-            stream=None) -> torch.Tensor:
+            stream=None, fused: bool = False) -> torch.Tensor:
         absorb_q(self.cfg, q_nope, w_uk, self.q_abs, stream)
         decode_attn(self.cfg, self.q_abs, q_rope, kv_cache, page_table, seqlens, max_pages,
                     self.workspace, stream)
-        splitkv_combine(self.cfg, self.workspace, self.batch, self.o_latent, self.lse, stream)
-        out_proj(self.cfg, self.o_latent, w_uv, self.out, stream)
+        if fused:
+            combine_out_proj(self.cfg, self.workspace, self.batch, w_uv, self.out, self.o_latent,
+                             self.lse, stream)
+        else:
+            splitkv_combine(self.cfg, self.workspace, self.batch, self.o_latent, self.lse, stream)
+            out_proj(self.cfg, self.o_latent, w_uv, self.out, stream)
         return self.out
 
 
 __all__ = [
     "Config", "make_config", "lib", "absorb_q", "workspace_size", "alloc_workspace",
-    "decode_attn", "splitkv_combine", "out_proj", "get_device_error", "decode_kernel_kind",
-    "decode_attn_noalloc",
+    "decode_attn", "splitkv_combine", "out_proj", "combine_out_proj", "get_device_error",
+    "decode_kernel_kind", "decode_attn_noalloc",
     "Decoder", "MlraError", "EXPORTS", "F32", "BF16",
 ]

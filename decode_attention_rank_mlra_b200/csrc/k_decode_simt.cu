@@ -37,6 +37,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   float* sc = sq + kHeadSlots * RS;         // [32][RS]  c_b | k_rope of the sub-tile
   float* sp = sc + kSub * RS;               // [16][32]  probabilities
 
+  pdl_wait();
+  pdl_trigger();
   const mlra_config_t& cfg = a.cfg;
   const int nb = cfg.n_blocks, H = cfg.n_heads, D = nb * DCB + DR;
   const int g = blockIdx.x / a.ctas_per_group;
@@ -184,8 +186,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t st) {
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int grid = a.n_groups * a.ctas_per_group;
-  kern<<<grid, kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, a);
 }
 
 }  // namespace

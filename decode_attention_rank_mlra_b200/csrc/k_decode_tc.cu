@@ -56,40 +56,6 @@ struct TcShape {
   static_assert(kStages >= 3, "too few pipeline stages");
 };
 
-struct Piece {
-  int s, t0, t1, slot, L;
-};
-
-// Walks the pieces (sequence, tile range) of one CTA's share of the tile stream.
-// Only the first piece needs a search; the next ones follow sequence by sequence.
-struct Walker {
-  const int32_t* tile_off;
-  const int32_t* slot_off;
-  const int32_t* seqlens;
-  int batch, share, cap, gt, end;
-  int cur = -1;
-  __device__ bool next(Piece& p) {
-    if (gt >= end) return false;
-    int s;
-    if (cur < 0) {
-      s = find_seq(tile_off, batch, gt);
-    } else {
-      s = cur + 1;
-      while (__ldg(tile_off + s + 1) <= gt) ++s;  // skip empty sequences
-    }
-    cur = s;
-    const int s0 = __ldg(tile_off + s), s1 = __ldg(tile_off + s + 1);
-    const int pe = min(end, s1);
-    p.s = s;
-    p.t0 = gt - s0;
-    p.t1 = pe - s0;
-    p.slot = __ldg(slot_off + s) + (gt / share - s0 / share);
-    p.L = min(max(__ldg(seqlens + s), 0), cap);
-    gt = pe;
-    return true;
-  }
-};
-
 // Bounded mbarrier wait: false on timeout (error recorded) or when another role aborted.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* err) {
@@ -169,6 +135,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   const char* wsc = static_cast<const char*>(a.ws);
   const int nb = a.cfg.n_blocks, H = a.cfg.n_heads;
@@ -179,7 +147,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int total = hdr->total_tiles, share = hdr->share;
   Walker walk{reinterpret_cast<const int32_t*>(wsc + a.L.tile_off),
               reinterpret_cast<const int32_t*>(wsc + a.L.slot_off),
-              a.seqlens, a.batch, share, a.cap, c * share, min(total, (c + 1) * share)};
+              a.seqlens,
+              reinterpret_cast<const CtaStart*>(wsc + a.L.cta_start) + c,
+              a.batch, a.cap, c * share, min(total, (c + 1) * share)};
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
@@ -571,8 +541,8 @@ cudaError_t launch_t(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t s
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<a.n_groups * a.ctas_per_group, kThreadsTC, S::kSmem, st>>>(map, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(a.n_groups * a.ctas_per_group), dim3(kThreadsTC), S::kSmem, st, map,
+                    a);
 }
 
 }  // namespace

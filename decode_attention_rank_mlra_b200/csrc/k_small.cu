@@ -45,9 +45,11 @@ __device__ int block_inclusive_scan(int v, int* warp_tot) {
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                     int cap, int ctas_per_group, int max_slots,
                                                     WsHeader* hdr, int32_t* tile_off,
-                                                    int32_t* slot_off) {
+                                                    int32_t* slot_off, CtaStart* cta_start) {
   __shared__ int warp_tot[32];
   __shared__ int s_total, s_share, s_bad;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x == 0) { hdr->error = 0; s_bad = 0; }
   __syncthreads();
   const int per = (batch + blockDim.x - 1) / blockDim.x;
@@ -78,7 +80,15 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   run = incl - local;
   for (int s = b0; s < b1; ++s) {
     slot_off[s] = run;
-    int a = tile_off[s], e = tile_off[s + 1];
+    const int a = tile_off[s], e = tile_off[s + 1];
+    // every CTA whose share starts inside this sequence
+    const int L = min(max(__ldg(seqlens + s), 0), cap);
+    for (int c = (a + share - 1) / share; c * share < e; ++c) {
+      CtaStart cs;
+      cs.s = s; cs.s0 = a; cs.s1 = e; cs.slot = run + c - a / share; cs.L = L;
+      cs.pad[0] = cs.pad[1] = cs.pad[2] = 0;
+      cta_start[c] = cs;
+    }
     run += (e > a) ? ((e - 1) / share - a / share + 1) : 0;
   }
   if (threadIdx.x == blockDim.x - 1) {
@@ -97,11 +107,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 cudaError_t launch_plan(const int32_t* seqlens, int batch, int cap, int ctas_per_group, void* ws,
                         const WsLayout& L, cudaStream_t st) {
   char* base = static_cast<char*>(ws);
-  plan_kernel<<<1, 1024, 0, st>>>(seqlens, batch, cap, ctas_per_group, L.max_slots,
-                                  reinterpret_cast<WsHeader*>(base),
-                                  reinterpret_cast<int32_t*>(base + L.tile_off),
-                                  reinterpret_cast<int32_t*>(base + L.slot_off));
-  return cudaGetLastError();
+  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, seqlens, batch, cap, ctas_per_group,
+                    L.max_slots, reinterpret_cast<WsHeader*>(base),
+                    reinterpret_cast<int32_t*>(base + L.tile_off),
+                    reinterpret_cast<int32_t*>(base + L.slot_off),
+                    reinterpret_cast<CtaStart*>(base + L.cta_start));
 }
 
 // ---------------------------------------------------------------------------
@@ -147,6 +157,8 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_kernel(const T* __restrict
                                                              const T* __restrict__ w_uk,
                                                              float* __restrict__ q_abs, int batch,
                                                              int heads, int nb, int d_cb, int d_h) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float4 sq4[];  // [kSeqBlk][d_h / 4]
   float* sq = reinterpret_cast<float*>(sq4);
   const int h = blockIdx.x, s0 = blockIdx.z * kSeqBlk;
@@ -196,14 +208,11 @@ cudaError_t launch_absorb(const mlra_config_t& c, const void* q_nope, const void
             (batch + kSeqBlk - 1) / kSeqBlk);
   size_t sm = sizeof(float) * kSeqBlk * c.d_h;
   if (c.dtype == MLRA_BF16)
-    absorb_kernel<__nv_bfloat16><<<grid, kAbsThreads, sm, st>>>(
-        (const __nv_bfloat16*)q_nope, (const __nv_bfloat16*)w_uk, q_abs, batch, c.n_heads,
-        c.n_blocks, c.d_cb, c.d_h);
-  else
-    absorb_kernel<float><<<grid, kAbsThreads, sm, st>>>((const float*)q_nope, (const float*)w_uk,
-                                                        q_abs, batch, c.n_heads, c.n_blocks,
-                                                        c.d_cb, c.d_h);
-  return cudaGetLastError();
+    return launch_pdl(absorb_kernel<__nv_bfloat16>, grid, dim3(kAbsThreads), sm, st,
+                      (const __nv_bfloat16*)q_nope, (const __nv_bfloat16*)w_uk, q_abs, batch,
+                      c.n_heads, c.n_blocks, c.d_cb, c.d_h);
+  return launch_pdl(absorb_kernel<float>, grid, dim3(kAbsThreads), sm, st, (const float*)q_nope,
+                    (const float*)w_uk, q_abs, batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h);
 }
 
 // ---------------------------------------------------------------------------
@@ -216,6 +225,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const char* __restrict__ w
                                                       int batch, int heads, int nb, int d_cb,
                                                       float* __restrict__ o_latent,
                                                       float* __restrict__ lse_out) {
+  pdl_wait();
+  pdl_trigger();
   const int warp_g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int total = batch * heads * nb;
@@ -279,9 +290,8 @@ cudaError_t launch_combine(const mlra_config_t& c, const void* ws, const WsLayou
   const int rows = batch * c.n_heads * c.n_blocks;
   const int blocks = (rows * 32 + 255) / 256;
   if (blocks == 0) return cudaSuccess;
-  combine_kernel<<<blocks, 256, 0, st>>>(static_cast<const char*>(ws), L, batch, c.n_heads,
-                                         c.n_blocks, c.d_cb, o_latent, lse);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const char*>(ws), L,
+                    batch, c.n_heads, c.n_blocks, c.d_cb, o_latent, lse);
 }
 
 // ---------------------------------------------------------------------------
@@ -311,6 +321,8 @@ __global__ void __launch_bounds__(kOpWarps * 32) out_proj_kernel(const float* __
                                                                  float* __restrict__ out, int batch,
                                                                  int heads, int nb, int d_cb,
                                                                  int d_h, float branch_scale) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float4 sm4[];
   const int K = nb * d_cb;
   float* so = reinterpret_cast<float*>(sm4);    // [K][kSeqBlk]
@@ -390,14 +402,12 @@ cudaError_t launch_out_proj(const mlra_config_t& c, const float* o_latent, const
     }
   }
   if (c.dtype == MLRA_BF16)
-    out_proj_kernel<__nv_bfloat16><<<grid, kOpWarps * 32, sm, st>>>(
-        o_latent, (const __nv_bfloat16*)w_uv, out, batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h,
-        c.branch_scale);
-  else
-    out_proj_kernel<float><<<grid, kOpWarps * 32, sm, st>>>(o_latent, (const float*)w_uv, out,
-                                                            batch, c.n_heads, c.n_blocks, c.d_cb,
-                                                            c.d_h, c.branch_scale);
-  return cudaGetLastError();
+    return launch_pdl(out_proj_kernel<__nv_bfloat16>, grid, dim3(kOpWarps * 32), sm, st, o_latent,
+                      (const __nv_bfloat16*)w_uv, out, batch, c.n_heads, c.n_blocks, c.d_cb,
+                      c.d_h, c.branch_scale);
+  return launch_pdl(out_proj_kernel<float>, grid, dim3(kOpWarps * 32), sm, st, o_latent,
+                    (const float*)w_uv, out, batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h,
+                    c.branch_scale);
 }
 
 }  // namespace mlra

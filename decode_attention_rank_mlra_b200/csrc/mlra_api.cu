@@ -66,6 +66,20 @@ int choose_kernel(const mlra_config_t& c, int dev) {
   return 0;
 }
 
+// Tensor-core absorption / output projection on this device for this config?
+// MLRA_PROJ_KERNEL=simt forces the SIMT kernels (tests cross-check both).
+bool use_proj_tc(const mlra_config_t& c) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* e = getenv("MLRA_PROJ_KERNEL");
+    forced = (e && strcmp(e, "simt") == 0) ? 1 : 0;
+  }
+  if (forced == 1 || !proj_tc_supported(c)) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  return device_is_sm100(dev);
+}
+
 struct Grid { int kind, n_groups, ctas_per_group; };
 
 mlra_status_t plan_grid(const mlra_config_t& c, Grid* g) {
@@ -80,7 +94,8 @@ mlra_status_t plan_grid(const mlra_config_t& c, Grid* g) {
 }
 
 WsLayout layout_for(const mlra_config_t& c, int batch, const Grid& g) {
-  return ws_layout(batch, c.n_heads, c.n_blocks, c.d_cb, batch + g.ctas_per_group);
+  return ws_layout(batch, c.n_heads, c.n_blocks, c.d_cb, batch + g.ctas_per_group,
+                   g.ctas_per_group);
 }
 
 mlra_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
@@ -122,6 +137,10 @@ mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const 
   if (!q_nope || !w_uk || !q_abs) return MLRA_ERR_INVALID_ARG;
   if (!aligned(w_uk, 16) || !aligned(q_nope, cfg->dtype == MLRA_BF16 ? 2 : 4) || !aligned(q_abs, 4))
     return MLRA_ERR_ALIGNMENT;
+  if (use_proj_tc(*cfg) && aligned(q_nope, 16)) {
+    cudaError_t e = launch_absorb_tc(*cfg, q_nope, w_uk, q_abs, batch, (cudaStream_t)stream);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+  }
   return from_cuda(launch_absorb(*cfg, q_nope, w_uk, q_abs, batch, (cudaStream_t)stream));
 }
 
@@ -210,7 +229,42 @@ mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_latent, con
   if (batch == 0) return MLRA_OK;
   if (!o_latent || !w_uv || !out) return MLRA_ERR_INVALID_ARG;
   if (!aligned(w_uv, 16) || !aligned(o_latent, 4) || !aligned(out, 4)) return MLRA_ERR_ALIGNMENT;
+  if (use_proj_tc(*cfg) && aligned(o_latent, 16)) {
+    WsLayout none{};
+    cudaError_t e = launch_out_proj_tc(*cfg, o_latent, nullptr, none, nullptr, nullptr, w_uv, out,
+                                       batch, (cudaStream_t)stream);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+  }
   return from_cuda(launch_out_proj(*cfg, o_latent, w_uv, out, batch, (cudaStream_t)stream));
+}
+
+mlra_status_t mlra_combine_out_proj(const mlra_config_t* cfg, const void* workspace,
+                                    size_t workspace_bytes, int32_t batch, const void* w_uv,
+                                    float* out, float* o_latent, float* lse,
+                                    mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0 || !workspace) return MLRA_ERR_INVALID_ARG;
+  if (batch == 0) return MLRA_OK;
+  if (!w_uv || !out) return MLRA_ERR_INVALID_ARG;
+  if (!aligned(w_uv, 16) || !aligned(out, 4) || (o_latent && !aligned(o_latent, 4)) ||
+      (lse && !aligned(lse, 4)))
+    return MLRA_ERR_ALIGNMENT;
+  Grid g;
+  st = plan_grid(*cfg, &g);
+  if (st != MLRA_OK) return st;
+  const WsLayout L = layout_for(*cfg, batch, g);
+  if (workspace_bytes < L.total) return MLRA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (use_proj_tc(*cfg) && (!o_latent || aligned(o_latent, 16))) {
+    cudaError_t e = launch_out_proj_tc(*cfg, nullptr, workspace, L, o_latent, lse,
+                                       w_uv, out, batch, s);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+  }
+  if (!o_latent) return MLRA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_combine(*cfg, workspace, L, batch, o_latent, lse, s);
+  if (e != cudaSuccess) return MLRA_ERR_CUDA;
+  return from_cuda(launch_out_proj(*cfg, o_latent, w_uv, out, batch, s));
 }
 
 mlra_status_t mlra_get_device_error(const void* workspace, size_t workspace_bytes,

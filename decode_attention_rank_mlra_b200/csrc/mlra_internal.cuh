@@ -19,6 +19,7 @@ constexpr int kPageSize = 64;
 //   Header                       256 B
 //   tile_off  [batch + 1] int32   first tile of each sequence in the tile stream
 //   slot_off  [batch + 1] int32   first split slot of each sequence
+//   cta_start [n_ctas] CtaStart   first piece of each persistent CTA's share
 //   o_part    [max_slots, h, nb, d_cb] fp32   normalised latent output of a split
 //   lse_part  [max_slots, h, nb]       fp32   natural-log sum of exp of a split
 // ---------------------------------------------------------------------------
@@ -34,22 +35,30 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header must be 256 bytes");
 
+// The piece a CTA starts with: sequence s, its tiles [s0, s1) in the stream,
+// the split slot of the CTA's part of s, and s's (clamped) length.
+struct CtaStart {
+  int32_t s, s0, s1, slot, L, pad[3];
+};
+
 struct WsLayout {
-  size_t tile_off, slot_off, o_part, lse_part, total;
-  int32_t max_slots;
+  size_t tile_off, slot_off, cta_start, o_part, lse_part, total;
+  int32_t max_slots, n_ctas;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline WsLayout ws_layout(int batch, int heads, int nb, int d_cb, int max_slots) {
+inline WsLayout ws_layout(int batch, int heads, int nb, int d_cb, int max_slots, int n_ctas) {
   WsLayout L;
   size_t off = sizeof(WsHeader);
-  L.tile_off = off; off = align256(off + sizeof(int32_t) * (batch + 1));
-  L.slot_off = off; off = align256(off + sizeof(int32_t) * (batch + 1));
-  L.o_part = off;   off = align256(off + sizeof(float) * size_t(max_slots) * heads * nb * d_cb);
-  L.lse_part = off; off = align256(off + sizeof(float) * size_t(max_slots) * heads * nb);
+  L.tile_off = off;  off = align256(off + sizeof(int32_t) * (batch + 1));
+  L.slot_off = off;  off = align256(off + sizeof(int32_t) * (batch + 1));
+  L.cta_start = off; off = align256(off + sizeof(CtaStart) * size_t(n_ctas));
+  L.o_part = off;    off = align256(off + sizeof(float) * size_t(max_slots) * heads * nb * d_cb);
+  L.lse_part = off;  off = align256(off + sizeof(float) * size_t(max_slots) * heads * nb);
   L.total = off;
   L.max_slots = max_slots;
+  L.n_ctas = n_ctas;
   return L;
 }
 
@@ -58,17 +67,8 @@ __device__ __forceinline__ void set_error(int32_t* err, int32_t code) {
   atomicCAS(err, 0, code);
 }
 
-// Split bookkeeping shared by the decode kernels: the tile stream of all
-// sequences is cut into `share`-tile pieces, one per CTA of a branch group.
-struct Plan {
-  const int32_t* tile_off;  // [batch+1]
-  const int32_t* slot_off;  // [batch+1]
-  const int32_t* seqlens;   // [batch]
-  int32_t batch;
-  int32_t total_tiles;
-  int32_t share;
-};
-
+// Split bookkeeping of the decode kernels: the tile stream of all sequences
+// is cut into `share`-tile pieces, one per CTA of a branch group.
 // Sequence containing global tile `t` (tile_off is non-decreasing).
 __device__ __forceinline__ int find_seq(const int32_t* tile_off, int batch, int t) {
   int lo = 0, hi = batch - 1;
@@ -77,6 +77,91 @@ __device__ __forceinline__ int find_seq(const int32_t* tile_off, int batch, int 
     if (__ldg(tile_off + mid) <= t) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// One piece of a CTA's share: tiles [t0, t1) of sequence s (tile indices
+// within the sequence), written to split slot `slot`; L = the sequence length.
+struct Piece {
+  int s, t0, t1, slot, L;
+};
+
+// Walks the pieces of one persistent CTA's share [gt, end) of the tile stream.
+// The first piece comes from the plan's per-CTA start record; each later piece
+// starts a new sequence, whose bounds are loaded one piece ahead.
+struct Walker {
+  const int32_t* tile_off;
+  const int32_t* slot_off;
+  const int32_t* seqlens;
+  const CtaStart* start;
+  int batch, cap, gt, end;
+  int cur = -1, cur_s1 = 0;
+  int n_s1 = 0, n_slot = 0, n_L = 0;  // sequence cur + 1, loaded ahead
+
+  __device__ void load_ahead() {
+    const int s = cur + 1;
+    if (s < batch) {
+      n_s1 = __ldg(tile_off + s + 1);
+      n_slot = __ldg(slot_off + s);
+      n_L = __ldg(seqlens + s);
+    }
+  }
+  __device__ bool next(Piece& p) {
+    if (gt >= end) return false;
+    int s, s0, s1, slot, L;
+    if (cur < 0) {
+      const int4 a = __ldg(reinterpret_cast<const int4*>(start));
+      s = a.x; s0 = a.y; s1 = a.z; slot = a.w;
+      L = __ldg(&start->L);
+    } else {
+      s = cur + 1;
+      s0 = cur_s1;  // == gt: a later piece opens its sequence (split 0)
+      if (n_s1 > gt) {
+        s1 = n_s1; slot = n_slot; L = n_L;
+      } else {  // empty sequences in between
+        while (__ldg(tile_off + s + 1) <= gt) ++s;
+        s0 = __ldg(tile_off + s);
+        s1 = __ldg(tile_off + s + 1);
+        slot = __ldg(slot_off + s);
+        L = __ldg(seqlens + s);
+      }
+    }
+    const int pe = min(end, s1);
+    p.s = s;
+    p.t0 = gt - s0;
+    p.t1 = pe - s0;
+    p.slot = slot;
+    p.L = min(max(L, 0), cap);
+    gt = pe;
+    cur = s;
+    cur_s1 = s1;
+    load_ahead();
+    return true;
+  }
+};
+
+// Programmatic dependent launch: every kernel of the library is launched so
+// that the next kernel on the stream may start its prologue early; each one
+// waits for its predecessor's completion (and memory) before its first global
+// access, and lets its dependents launch right after.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... K, typename... A>
+cudaError_t launch_pdl(void (*kern)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<A&&>(args)...);
 }
 
 // Dispatch entry points of the individual kernel files (host side).
@@ -105,6 +190,15 @@ struct DecodeArgs {
   int32_t ctas_per_group;
   int32_t n_groups;
 };
+
+// Tensor-core absorption and output projection (bf16, d_h = 128).
+bool proj_tc_supported(const mlra_config_t& c);
+cudaError_t launch_absorb_tc(const mlra_config_t& c, const void* q_nope, const void* w_uk,
+                             float* q_abs, int batch, cudaStream_t st);
+cudaError_t launch_out_proj_tc(const mlra_config_t& c, const float* o_latent_in, const void* ws,
+                               const WsLayout& L, float* o_latent_out,
+                               float* lse_out, const void* w_uv, float* out, int batch,
+                               cudaStream_t st);
 
 // fp32 SIMT decode (any supported shape / dtype).
 bool simt_supported(const mlra_config_t& c);

@@ -170,6 +170,26 @@ MLRA_API mlra_status_t mlra_out_proj(const mlra_config_t* cfg, const float* o_la
                             float* out, int32_t batch, mlra_stream_t stream);
 
 /*
+ * Steps 2b + 3 in one launch: the split partials of the workspace are merged
+ * (as mlra_splitkv_combine) while they are staged as the operand of the output
+ * up-projection (as mlra_out_proj).  The paper describes the two steps, not
+ * their fusion; the result is the same up to fp32 rounding order.
+ *   workspace : the one passed to the preceding mlra_decode_attn (same stream)
+ *   w_uv      : [n_blocks, n_heads, d_cb, d_h] dtype, 16-byte aligned
+ *   out       : [batch, n_heads, d_h] fp32 (written)
+ *   o_latent  : [batch, n_heads, n_blocks, d_cb] fp32, written when not NULL
+ *               (16-byte aligned)
+ *   lse       : [batch, n_heads, n_blocks] fp32, written when not NULL
+ * Runs as one tensor-core kernel for bf16 with d_h = 128, d_cb a multiple of
+ * 128 and n_blocks * d_cb <= 512 on sm_100; otherwise it runs the two steps
+ * one after the other, which needs o_latent (MLRA_ERR_UNSUPPORTED if NULL).
+ */
+MLRA_API mlra_status_t mlra_combine_out_proj(const mlra_config_t* cfg, const void* workspace,
+                                    size_t workspace_bytes, int32_t batch, const void* w_uv,
+                                    float* out, float* o_latent, float* lse,
+                                    mlra_stream_t stream);
+
+/*
  * Read (and then clear) the device error word of a workspace.  Synchronises
  * `stream`.  *device_status receives MLRA_OK or the first device-side error
  * (MLRA_ERR_BAD_PAGE, MLRA_ERR_TIMEOUT) recorded since the last decode call.

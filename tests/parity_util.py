@@ -25,14 +25,16 @@ def config_of(spec: W.WorkloadSpec) -> mlra.Config:
                             branch_scale=spec.branch_scale)
 
 
-def run_gpu(inp: W.DecodeInputs) -> Dict[str, torch.Tensor]:
-    """Full decode step through the C ABI; returns CPU copies of every output."""
+def run_gpu(inp: W.DecodeInputs, fused: bool = False) -> Dict[str, torch.Tensor]:
+    """Full decode step through the C ABI; returns CPU copies of every output.
+
+    ``fused``: merge + projection through mlra_combine_out_proj."""
     spec = inp.spec
     cfg = config_of(spec)
     dec = mlra.Decoder(cfg, spec.batch, inp.device)
     max_pages = inp.page_table.shape[1] if inp.page_table is not None else inp.max_len
     dec.run(inp.q_nope, inp.q_rope, inp.w_uk, inp.w_uv, inp.kv_cache, inp.page_table,
-            inp.seqlens, max_pages)
+            inp.seqlens, max_pages, fused=fused)
     err = mlra.get_device_error(dec.workspace)
     torch.cuda.synchronize()
     return dict(out=dec.out.cpu(), o_lat=dec.o_latent.cpu(), lse=dec.lse.cpu(),

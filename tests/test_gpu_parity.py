@@ -42,25 +42,57 @@ def test_fp32_workload_full():
     check_close(got["q_abs"][0].double().numpy(), qa, "f32", "q_abs")
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("name,seqlens", [
     ("mlra4_bf16_b16_h16_l4096_contig", [1, 63, 64, 65, 700, 1500]),
     ("mlra4_bf16_b64_h32_l16384_paged", [129, 1000, 2049]),
     ("mlra4_bf16_b128_h16_ragged1k_64k_paged", [1, 64, 333, 1024, 2500, 77]),
 ])
-def test_bf16_oracle_sized(name, seqlens):
+def test_bf16_oracle_sized(name, seqlens, fused):
     inp = _small(name, len(seqlens), seqlens)
-    got = run_gpu(inp)
+    got = run_gpu(inp, fused=fused)
     assert got["device_error"] == 0
     compare_batch(inp, got)
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("name", ["mla_bf16_b8_h128_l131072_paged",
                                   "mlra4_bf16_b8_h128_l131072_paged"])
-def test_bf16_h128_oracle_sized(name):
+def test_bf16_h128_oracle_sized(name, fused):
     inp = _small(name, 2, [1100, 190])
-    got = run_gpu(inp)
+    got = run_gpu(inp, fused=fused)
     assert got["device_error"] == 0
     compare_batch(inp, got, heads=[0, 1, 63, 100, 127])
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("batch", [17, 70, 300])
+def test_batches_spanning_several_sequence_tiles(batch, fused):
+    """Batches that fill several N tiles of the weight contractions (16..256
+    sequences per CTA) with a partial last tile, and many short sequences."""
+    rng = np.random.default_rng(batch)
+    seqlens = rng.integers(0, 150, size=batch)
+    seqlens[0] = 150
+    inp = _small("mlra4_bf16_b64_h32_l16384_paged", batch, seqlens)
+    got = run_gpu(inp, fused=fused)
+    assert got["device_error"] == 0
+    pick = sorted({0, 1, batch // 2, batch - 17, batch - 1})
+    compare_batch(inp, got, seqs=pick, heads=[0, 13, 31])
+
+
+def test_fused_projection_without_latent_outputs():
+    """combine_out_proj with o_latent = lse = None gives the same out."""
+    inp = _small("mlra4_bf16_b16_h16_l4096_contig", 3, [500, 64, 1])
+    ref = run_gpu(inp, fused=True)
+    spec = inp.spec
+    cfg = config_of(spec)
+    dec = mlra.Decoder(cfg, spec.batch, inp.device)
+    mlra.absorb_q(cfg, inp.q_nope, inp.w_uk, dec.q_abs)
+    mlra.decode_attn(cfg, dec.q_abs, inp.q_rope, inp.kv_cache, None, inp.seqlens, inp.max_len,
+                     dec.workspace)
+    out = mlra.combine_out_proj(cfg, dec.workspace, spec.batch, inp.w_uv)
+    torch.cuda.synchronize()
+    assert torch.equal(out.cpu(), ref["out"])
 
 
 def test_empty_and_single_token_sequences():
@@ -188,7 +220,7 @@ FULL = [
 def test_full_size_sampled(name, samples):
     spec = W.WORKLOADS[name]
     inp = W.make_inputs(spec, "cuda")
-    got = run_gpu(inp)
+    got = run_gpu(inp, fused=True)
     assert got["device_error"] == 0
     assert torch.all(torch.isfinite(got["out"]))
     L_all = inp.seqlens.cpu().numpy()
