@@ -125,6 +125,8 @@ def cpu_baseline(spec, seconds: float):
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi sampling every 25 ms in one long-running process; each line is
+    stamped with the host clock when it arrives."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -132,29 +134,36 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.samples = []
-        self._stop = threading.Event()
+        self._proc = None
         self._th = None
 
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                out = subprocess.run(
-                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                     "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-                if out.returncode == 0 and out.stdout.strip():
-                    self.samples.append((time.perf_counter(), out.stdout.strip().split(", ")))
-            except Exception:
-                pass
-            self._stop.wait(0.2)
+    def _read(self):
+        for line in self._proc.stdout:
+            line = line.strip()
+            if line:
+                self.samples.append((time.perf_counter(), [x.strip() for x in line.split(",")]))
 
     def start(self):
-        self._th = threading.Thread(target=self._run, daemon=True)
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "25"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self._proc = None
+            return
+        self._th = threading.Thread(target=self._read, daemon=True)
         self._th.start()
 
     def stop(self):
-        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
         if self._th:
-            self._th.join(timeout=10)
+            self._th.join(timeout=5)
 
     def summary(self, t0: float, t1: float):
         inside = [s for t, s in self.samples if t0 <= t <= t1]
@@ -169,6 +178,48 @@ class ClockSampler:
         return {"sm_mhz": float(np.median(sm)) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over the process group (identity
+    on one rank).  Every rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def aggregate_rate(world: int, batch: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank decodes `batch` sequences per step (weak
+    scaling, independent replicas); the step time is the slowest rank's."""
+    return world * batch / (ms_per_step * 1e-3)
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu capture, or None.
+
+    The figure is used only while the attention kernel's sources are the ones
+    it was measured on (their sha256 is stored beside it).
+    """
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        h = hashlib.sha256()
+        csrc = os.path.join(ROOT, "decode_attention_rank_mlra_b200", "csrc")
+        for name in ("k_decode_tc.cu", "sm100_ptx.cuh", "mlra_internal.cuh"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != t["sources_sha256"]:
+            return None, "kernel changed since the ncu capture"
+        w = t["workloads"].get(workload)
+        if w is None:
+            return None, "no ncu capture for this workload"
+        return int(w["dram_bytes_per_launch"]), w["profile"]
+    except Exception as e:  # pragma: no cover
+        return None, f"unavailable ({type(e).__name__})"
 
 
 def measured_peak():
@@ -338,14 +389,12 @@ def run_ours(args):
         raise RuntimeError("device error during timing")
 
     # max over ranks
-    vals = torch.tensor([ms_total, e2e_ms, float(np.mean(k_ms))], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms, k_mean = [float(v) for v in vals.cpu()]
+    ms_total, e2e_ms, k_mean = max_over_ranks([ms_total, e2e_ms, float(np.mean(k_ms))], dev)
     ms_step = ms_total / args.steps
-    value = world * B / (ms_step * 1e-3)
+    value = aggregate_rate(world, B, ms_step)
     peak, peak_kind = measured_peak()
     achieved = cache_bytes / (k_mean * 1e-3) / 1e9
+    traffic, traffic_src = measured_traffic(spec.name) if kind == "tcgen05" else (None, "SIMT kernel")
     result = None
     if rank == 0:
         clocks = sampler.summary(t_wall0, t_wall1)
@@ -366,13 +415,13 @@ def run_ours(args):
             "hbm_gbs_step": cache_bytes / (ms_step * 1e-3) / 1e9,
             "roofline": {
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
                 "kernel": "mlra_decode_attn (plan + attention kernel): one CUDA-graph launch per event pair on the launch stream, K launches",
                 "algorithmic_bytes_per_launch": cache_bytes,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
             },
-            "e2e": {"value": world * B / (e2e_ms / e2e_steps * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": aggregate_rate(world, B, e2e_ms / e2e_steps), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(h_qn.numel() * h_qn.element_size()
                                               + h_qr.numel() * h_qr.element_size()
                                               + h_sl.numel() * h_sl.element_size()),

@@ -1,0 +1,77 @@
+"""The bench's multi-rank plumbing on CPU: two gloo ranks, max over ranks,
+whole-job aggregation, and rank-0-only output of the reference arm."""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out_dir: str):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        # rank r took (r + 1) ms in total and 10 - r ms end to end
+        got = bench.max_over_ranks([rank + 1.0, 10.0 - rank, 0.5 * rank])
+        dist.barrier()
+        with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+            f.write(",".join(repr(v) for v in got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_two_gloo_ranks(tmp_path):
+    world, port = 2, _free_port()
+    mp.start_processes(_rank_main, args=(world, port, str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    for r in range(world):
+        vals = [float(x) for x in (tmp_path / f"rank{r}.txt").read_text().split(",")]
+        assert vals == [2.0, 10.0, 0.5]
+
+
+def test_single_rank_is_identity():
+    import bench
+    assert not dist.is_initialized()
+    assert bench.max_over_ranks([3.0, 1.5]) == [3.0, 1.5]
+
+
+def test_aggregate_is_whole_job_weak_scaling():
+    import bench
+    # 8 replicas x 16 sequences each, 0.05 ms per step (slowest rank)
+    assert bench.aggregate_rate(8, 16, 0.05) == pytest.approx(8 * 16 / 0.05e-3)
+    assert bench.aggregate_rate(1, 16, 0.05) * 8 == pytest.approx(bench.aggregate_rate(8, 16, 0.05))
+
+
+def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
+    import bench
+
+    class Args:
+        workload = "mlra4_f32_b1_h4_l256"
+        steps = 1
+        warmup = 0
+        impl = "reference"
+
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.run_reference(Args()) is None
+    monkeypatch.setenv("RANK", "0")
+    res = bench.run_reference(Args())
+    assert res["impl"] == "reference" and res["value"] > 0
+    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["cpu_baseline"]["kind"] == "oracle"
