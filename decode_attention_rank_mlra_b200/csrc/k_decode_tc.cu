@@ -38,10 +38,12 @@ constexpr int kBoxCols = 64;                 // bf16 columns per TMA box (128 B)
 constexpr int kBoxBytes = kTile * 128;       // 64 rows x 128 B
 constexpr int kThreadsTC = 192;              // warps 0-3 softmax, 4 TMA, 5 MMA
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQ = 0;                // q_abs rows (bf16 pairs): 64 columns
-constexpr uint32_t kColQr = 64;              // q_rope rows: 32 columns
-constexpr uint32_t kColS = 128;              // S / P double buffer: 2 x 64 columns
-constexpr uint32_t kColO = 256;              // O accumulator: 128 columns
+// Queries are double-buffered by piece: buffer b at b * kQBuf holds the q_abs
+// rows (bf16 pairs, 64 columns) and then the q_rope rows (32 columns).
+constexpr uint32_t kQBuf = 96;
+constexpr uint32_t kColQr = 64;              // q_rope offset inside a query buffer
+constexpr uint32_t kColS = 2 * kQBuf;        // S / P double buffer: 2 x 64 columns
+constexpr uint32_t kColO = kColS + 128;      // O accumulator: 128 columns
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kSmemLimit = 232448;           // max dynamic shared memory per block
 
@@ -51,7 +53,7 @@ struct TcShape {
   static constexpr int kStage = kBoxes * kBoxBytes;
   static constexpr int kStagesRaw = (kSmemLimit - 2048) / kStage;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kBars = 2 * kStages + 8;
+  static constexpr int kBars = 2 * kStages + 9;
   static constexpr int kSmem = 1024 + kStages * kStage + kBars * 8 + 64;
   static_assert(kStages >= 3, "too few pipeline stages");
 };
@@ -105,8 +107,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   // PV of tile k commits to PVDONE(k & 1): a waiter for PV(k) has always seen
   // S(k) or later, which implies PV(k-2) is complete, so parity waits are exact.
   auto PVDONE = [&](int i) { return bar0 + 8u * (2 * NST + 4 + i); };
-  const uint32_t QREADY = bar0 + 8u * (2 * NST + 6);
-  const uint32_t DRAIN = bar0 + 8u * (2 * NST + 7);
+  auto QREADY = [&](int i) { return bar0 + 8u * (2 * NST + 6 + i); };
+  const uint32_t DRAIN = bar0 + 8u * (2 * NST + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
@@ -122,7 +124,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(PREADY(i), 4);
       mbar_init(PVDONE(i), 1);
     }
-    mbar_init(QREADY, 4);
+    mbar_init(QREADY(0), 4);
+    mbar_init(QREADY(1), 4);
     mbar_init(DRAIN, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -235,7 +238,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mma_commit_warp(PVDONE(pit & 1));
     };
     while (ok && walk.next(p)) {
-      if (!wait_bar(QREADY, piece & 1, abort_flag, err)) { ok = false; break; }
+      if (!wait_bar(QREADY(piece & 1), (piece >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      const uint32_t qbuf = tmem + uint32_t(piece & 1) * kQBuf;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int st = it % NST, sb = it & 1;
         if (!wait_bar(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             if (g * G + bx >= nb) continue;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              mma_ts_warp(s_acc, tmem + kColQ + 8 * k,
+              mma_ts_warp(s_acc, qbuf + 8 * k,
                           d + uint64_t(((2 * bx + (k >> 2)) * kBoxBytes + (k & 3) * 32) >> 4),
                           kIdescQK, k > 0 ? 1u : 0u, (0 / WPB == bx) ? 0u : ~0u,
                           (1 / WPB == bx) ? 0u : ~0u, (2 / WPB == bx) ? 0u : ~0u,
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_ts_warp(s_acc, tmem + kColQr + 8 * k,
+            mma_ts_warp(s_acc, qbuf + kColQr + 8 * k,
                         d + uint64_t((2 * G * kBoxBytes + k * 32) >> 4), kIdescQK, 1u, 0u, 0u, 0u,
                         0u);
           mma_commit_warp(SFULL(sb));
@@ -281,6 +285,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         prev = it;
         prev_first = (t == p.t0);
+      }
+      // the piece's last PV goes out before the next piece's first QK: the
+      // epilogue waits for it, and must not wait for the next piece's data
+      if (ok && prev >= 0) {
+        if (!wait_bar(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(prev, prev_first);
+        prev = -1;
       }
       ++piece;
     }
@@ -322,37 +334,54 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     auto qr_row = [&](const Piece& pc) {
       return reinterpret_cast<const uint4*>(q_rope + (size_t(pc.s) * H + head) * 64);
     };
-    auto write_q = [&](const Piece& pc) {
-      uint32_t r[32];
-      const float4* q = q_row(pc);
+    // Lanes 0-15 of the quadrant hold the hi rows and lanes 16-31 the lo rows of
+    // the same 16 heads.  The .16x32bx2 TMEM accesses give thread t (< 16) both
+    // rows of head t for tokens 0-31 and thread t + 16 both rows for tokens
+    // 32-63, so S_hi + S_lo, the P_hi / P_lo write-back and O_hi + O_lo need no
+    // shuffles.
+    const uint32_t hi_t = row_t;                   // lane base 0 of the quadrant
+    const uint32_t lo_t = row_t + (16u << 16);     // lane base 16
+    // Queries of a piece into query buffer `buf`: thread t (x = 0) converts the
+    // first half of head t's row, thread t + 16 the second half, and the
+    // .16x32bx2 stores put the hi parts in the hi row and the lo parts in the
+    // lo row (the lo row's RoPE columns are zero).
+    auto write_q = [&](const Piece& pc, int buf) {
+      const float4* q = q_row(pc) + 16 * x;
+      float4 f[16];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float4 f[16];
+      for (int j = 0; j < 16; ++j) f[j] = active ? __ldg(q + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const uint4* qr = qr_row(pc) + 4 * x;
+      uint4 u[4];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) f[j] = active ? __ldg(q + 16 * half + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < 4; ++j) u[j] = active ? __ldg(qr + j) : make_uint4(0u, 0u, 0u, 0u);
+      uint32_t hi[32], lo[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float v[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
-          if (x) {  // lo part: what the bf16 hi part leaves out
+      for (int j = 0; j < 16; ++j) {
+        const float v[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
+        float w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] -= __bfloat162float(__float2bfloat16_rn(v[e]));
-          }
-          r[2 * j] = pack_bf16(v[0], v[1]);
-          r[2 * j + 1] = pack_bf16(v[2], v[3]);
-        }
-        tmem_st32(row_t + kColQ + 32 * half, r);
+        for (int e = 0; e < 4; ++e) w[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
+        hi[2 * j] = pack_bf16(v[0], v[1]);
+        hi[2 * j + 1] = pack_bf16(v[2], v[3]);
+        lo[2 * j] = pack_bf16(w[0], w[1]);
+        lo[2 * j + 1] = pack_bf16(w[2], w[3]);
       }
-      const uint4* qr = qr_row(pc);
+      const uint32_t qb = uint32_t(buf) * kQBuf;
+      tmem_st_x2_32<32>(hi_t + qb, hi);
+      tmem_st_x2_32<32>(lo_t + qb, lo);
+      uint32_t rr[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 u = (active && x == 0) ? __ldg(qr + j) : make_uint4(0u, 0u, 0u, 0u);
-        r[4 * j] = u.x; r[4 * j + 1] = u.y; r[4 * j + 2] = u.z; r[4 * j + 3] = u.w;
+      for (int j = 0; j < 4; ++j) {
+        rr[4 * j] = u[j].x; rr[4 * j + 1] = u[j].y; rr[4 * j + 2] = u[j].z; rr[4 * j + 3] = u[j].w;
       }
-      tmem_st32(row_t + kColQr, r);
+      tmem_st_x2_16<16>(hi_t + qb + kColQr, rr);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) rr[j] = 0u;
+      tmem_st_x2_16<16>(lo_t + qb + kColQr, rr);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(QREADY);
+      if (lane == 0) mbar_arrive(QREADY(buf));
     };
     // pull the next piece's query rows into L2 while this piece streams
     auto prefetch_q = [&](const Piece& pc) {
@@ -362,19 +391,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       prefetch_l2_evict_last(q + 256 * x + 128);
       if (x == 0) prefetch_l2_evict_last(qr_row(pc));
     };
-    // Lanes 0-15 of the quadrant hold the hi rows and lanes 16-31 the lo rows of
-    // the same 16 heads.  The .16x32bx2 TMEM accesses give thread t (< 16) both
-    // rows of head t for tokens 0-31 and thread t + 16 both rows for tokens
-    // 32-63, so S_hi + S_lo, the P_hi / P_lo write-back and O_hi + O_lo need no
-    // shuffles.
-    const uint32_t hi_t = row_t;                   // lane base 0 of the quadrant
-    const uint32_t lo_t = row_t + (16u << 16);     // lane base 16
     Piece p, pn;
-    int it = 0;
+    int it = 0, pidx = 0;
     bool ok = walk.next(p);
     bool has_next = ok && walk.next(pn);
-    if (ok) write_q(p);
-    if (has_next) prefetch_q(pn);
+    // the first two pieces' queries go in before the cache stream saturates
+    // memory; piece k + 1's go in during piece k's first tile (k >= 1)
+    if (ok) write_q(p, 0);
+    if (has_next) write_q(pn, 1);
     while (ok) {
       // m: the reference point of the exponentials, in log2 units.  It is the
       // first tile's max and moves only when a later tile would overflow
@@ -393,8 +417,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) raw[k] = __uint_as_float(sh[k]) + __uint_as_float(sl[k]);
         }
-        // every QK of this piece is done: the next piece's queries can go in now
-        if (t + 1 == p.t1 && has_next) write_q(pn);
         const int valid = min(kTile, p.L - t * kTile);
         if (valid < kTile) {
 #pragma unroll
@@ -462,6 +484,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(PREADY(sb));
+        // every QK of the previous piece is done: its query buffer takes the next piece's
+        if (t == p.t0 && pidx >= 1 && has_next) write_q(pn, (pidx + 1) & 1);
       }
       if (!ok) break;
       // ---- epilogue: o = (O_hi + O_lo) / l, lse
@@ -481,13 +505,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tmem_ld_x2_32<64>(lo_t + kColO + 32 * j, ol);
         tmem_wait_ld();
         if (active) {
-          float4* d4 = reinterpret_cast<float4*>(dst + 64 * x + 32 * j);
+          // 32-byte stores: each one fills a whole sector
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            d4[k] = make_float4((__uint_as_float(oh[4 * k]) + __uint_as_float(ol[4 * k])) * inv,
-                                (__uint_as_float(oh[4 * k + 1]) + __uint_as_float(ol[4 * k + 1])) * inv,
-                                (__uint_as_float(oh[4 * k + 2]) + __uint_as_float(ol[4 * k + 2])) * inv,
-                                (__uint_as_float(oh[4 * k + 3]) + __uint_as_float(ol[4 * k + 3])) * inv);
+          for (int k = 0; k < 4; ++k) {
+            float o8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              o8[e] = (__uint_as_float(oh[8 * k + e]) + __uint_as_float(ol[8 * k + e])) * inv;
+            st_global_v8(dst + 64 * x + 32 * j + 8 * k, o8);
+          }
         }
       }
       if (active && x == 0)
@@ -495,6 +521,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             l_tot > 0.f ? (m + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
       if (!has_next) break;
       p = pn;
+      ++pidx;
       has_next = walk.next(pn);
       if (has_next) prefetch_q(pn);
     }

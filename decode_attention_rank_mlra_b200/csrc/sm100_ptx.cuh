@@ -172,6 +172,15 @@ __device__ __forceinline__ void tmem_st_x2_16(uint32_t taddr, const uint32_t (&r
       MLRA_W8(0), MLRA_W8(8)
       : "memory");
 }
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st_x2_32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, {%2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32, %33};" ::"r"(taddr), "n"(SPLIT),
+      MLRA_W8(0), MLRA_W8(8), MLRA_W8(16), MLRA_W8(24)
+      : "memory");
+}
 #undef MLRA_R8
 #undef MLRA_W8
 
@@ -243,6 +252,13 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
       : "memory");
+}
+
+// 32-byte store of eight fp32 (full sector; the address is 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(float* p, const float (&v)[8]) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(v[0]),
+               "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
 }
 
 // ---- clusters / distributed shared memory -----------------------------------
