@@ -138,7 +138,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();
+  // No wait for the plan kernel launched just before: this kernel starts only
+  // after that kernel passed its own griddepcontrol.wait (so the queries, the
+  // lengths, the page table and the cache are final) and reset the error word;
+  // the CTA plans its first two pieces itself.
   pdl_trigger();
 
   const char* wsc = static_cast<const char*>(a.ws);
@@ -147,11 +150,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int c = blockIdx.x % a.ctas_per_group;
   const int g = grp % (nb / G);            // branch group
   const int head0 = (grp / (nb / G)) * HPC;  // first head of this CTA's head group
-  const int total = hdr->total_tiles, share = hdr->share;
+  __shared__ int plan_sm[12], scan_sm[kThreadsTC / 32 + 1];
+  plan_first_pieces<kThreadsTC>(a.seqlens, a.batch, a.cap, a.ctas_per_group, c, plan_sm, scan_sm);
+  const int total = plan_sm[0], share = plan_sm[1];
   Walker walk{reinterpret_cast<const int32_t*>(wsc + a.L.tile_off),
               reinterpret_cast<const int32_t*>(wsc + a.L.slot_off),
-              a.seqlens,
-              reinterpret_cast<const CtaStart*>(wsc + a.L.cta_start) + c,
+              a.seqlens, plan_sm + 2,
               a.batch, a.cap, c * share, min(total, (c + 1) * share)};
 
   if (warp == 4) {
@@ -529,6 +533,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   tc_fence_before();
   __syncthreads();
+  pdl_wait();  // complete only after the plan kernel (whose records the merge reads)
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

@@ -45,13 +45,19 @@ __device__ int block_inclusive_scan(int v, int* warp_tot) {
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                     int cap, int ctas_per_group, int max_slots,
                                                     WsHeader* hdr, int32_t* tile_off,
-                                                    int32_t* slot_off, CtaStart* cta_start) {
+                                                    int32_t* slot_off) {
   __shared__ int warp_tot[32];
   __shared__ int s_total, s_share, s_bad;
   pdl_wait();
-  pdl_trigger();
-  if (threadIdx.x == 0) { hdr->error = 0; s_bad = 0; }
+  // the error word is clear before the dependent attention kernel can start
+  // (it does not wait for this kernel and may record an error at once)
+  if (threadIdx.x == 0) {
+    hdr->error = 0;
+    __threadfence();
+    s_bad = 0;
+  }
   __syncthreads();
+  pdl_trigger();
   const int per = (batch + blockDim.x - 1) / blockDim.x;
   const int b0 = min(batch, (int)threadIdx.x * per), b1 = min(batch, b0 + per);
   auto tiles_of = [&](int s) {
@@ -81,14 +87,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   for (int s = b0; s < b1; ++s) {
     slot_off[s] = run;
     const int a = tile_off[s], e = tile_off[s + 1];
-    // every CTA whose share starts inside this sequence
-    const int L = min(max(__ldg(seqlens + s), 0), cap);
-    for (int c = (a + share - 1) / share; c * share < e; ++c) {
-      CtaStart cs;
-      cs.s = s; cs.s0 = a; cs.s1 = e; cs.slot = run + c - a / share; cs.L = L;
-      cs.pad[0] = cs.pad[1] = cs.pad[2] = 0;
-      cta_start[c] = cs;
-    }
     run += (e > a) ? ((e - 1) / share - a / share + 1) : 0;
   }
   if (threadIdx.x == blockDim.x - 1) {
@@ -110,8 +108,7 @@ cudaError_t launch_plan(const int32_t* seqlens, int batch, int cap, int ctas_per
   return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, seqlens, batch, cap, ctas_per_group,
                     L.max_slots, reinterpret_cast<WsHeader*>(base),
                     reinterpret_cast<int32_t*>(base + L.tile_off),
-                    reinterpret_cast<int32_t*>(base + L.slot_off),
-                    reinterpret_cast<CtaStart*>(base + L.cta_start));
+                    reinterpret_cast<int32_t*>(base + L.slot_off));
 }
 
 // ---------------------------------------------------------------------------

@@ -94,8 +94,7 @@ mlra_status_t plan_grid(const mlra_config_t& c, Grid* g) {
 }
 
 WsLayout layout_for(const mlra_config_t& c, int batch, const Grid& g) {
-  return ws_layout(batch, c.n_heads, c.n_blocks, c.d_cb, batch + g.ctas_per_group,
-                   g.ctas_per_group);
+  return ws_layout(batch, c.n_heads, c.n_blocks, c.d_cb, batch + g.ctas_per_group);
 }
 
 mlra_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
