@@ -23,19 +23,20 @@
 // Precision: queries and probabilities are carried as bf16 hi + lo pairs (two
 // MMA rows per head), so both enter the fp32-accumulated products with about
 // 16 significant bits while the cache stays the bf16 it is stored as.
-#include "mlra_internal.cuh"
-#include "sm100_ptx.cuh"
+#include "tc_common.cuh"
 
-#include <cudaTypedefs.h>
 #include <math.h>
 
 namespace mlra {
 namespace {
 
 using namespace ptx;
+using tc::kBoxBytes;
+using tc::kBoxCols;
+using tc::kSmemLimit;
+using tc::pack_bf16;
+using tc::wait_bar;
 
-constexpr int kBoxCols = 64;                 // bf16 columns per TMA box (128 B)
-constexpr int kBoxBytes = kTile * 128;       // 64 rows x 128 B
 constexpr int kThreadsTC = 192;              // warps 0-3 softmax, 4 TMA, 5 MMA
 constexpr uint32_t kTmemCols = 512;
 // Queries are double-buffered by piece: buffer b at b * kQBuf holds the q_abs
@@ -44,8 +45,6 @@ constexpr uint32_t kQBuf = 96;
 constexpr uint32_t kColQr = 64;              // q_rope offset inside a query buffer
 constexpr uint32_t kColS = 2 * kQBuf;        // S / P double buffer: 2 x 64 columns
 constexpr uint32_t kColO = kColS + 128;      // O accumulator: 128 columns
-constexpr uint64_t kTimeoutNs = 2000000000ull;
-constexpr int kSmemLimit = 232448;           // max dynamic shared memory per block
 
 template <int G>
 struct TcShape {
@@ -57,29 +56,6 @@ struct TcShape {
   static constexpr int kSmem = 1024 + kStages * kStage + kBars * 8 + 64;
   static_assert(kStages >= 3, "too few pipeline stages");
 };
-
-// Bounded mbarrier wait: false on timeout (error recorded) or when another role aborted.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int32_t* err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
-      set_error(err, MLRA_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
-  return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // G branches x HPC heads per CTA (rows = G * HPC * 2 <= 128).  The grid is
 // (branch groups x head groups) x CTAs per group; one CTA per SM.
@@ -540,19 +516,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 // Heads per CTA (a head group) and branches per CTA: the 128 MMA rows hold
 // G branches x HPC heads x (hi, lo).
 int hpc_of(const mlra_config_t& c) { return c.n_heads < 64 ? c.n_heads : 64; }
@@ -580,34 +543,25 @@ cudaError_t launch_t(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t s
 }  // namespace
 
 bool tc_supported(const mlra_config_t& c) {
-  if (c.dtype != MLRA_BF16 || c.d_cb != 128 || c.d_r != 64) return false;
+  if (c.dtype != MLRA_BF16 || c.d_r != 64) return false;
+  if (c.d_cb == 512) return tc::mla_supported(c);
+  if (c.d_cb != 128) return false;
   if (c.n_heads != 16 && c.n_heads != 32 && c.n_heads != 64 && c.n_heads != 128) return false;
   if (c.n_blocks != 1 && c.n_blocks != 2 && c.n_blocks != 4) return false;
   return c.n_blocks % g_of(c) == 0;
 }
 
 void tc_grid(const mlra_config_t& c, int num_sms, int* n_groups, int* ctas_per_group) {
-  *n_groups = (c.n_blocks / g_of(c)) * (c.n_heads / hpc_of(c));
+  *n_groups = c.d_cb == 512 ? tc::mla_groups(c) : (c.n_blocks / g_of(c)) * (c.n_heads / hpc_of(c));
   *ctas_per_group = num_sms / *n_groups > 0 ? num_sms / *n_groups : 1;
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   const mlra_config_t& c = a.cfg;
-  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
-  const int D = c.n_blocks * c.d_cb + c.d_r;
-  const uint64_t rows = a.page_table ? uint64_t(a.num_pages) * kPageSize
-                                     : uint64_t(a.batch) * uint64_t(a.max_pages);
-  if (rows >= (uint64_t(1) << 31)) return cudaErrorInvalidValue;
   CUtensorMap map;
-  cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
-  cuuint64_t strides[1] = {cuuint64_t(D) * 2};
-  cuuint32_t box[2] = {kBoxCols, kTile};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.kv_cache), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  cudaError_t e = tc::make_cache_map(a, &map);
+  if (e != cudaSuccess) return e;
+  if (c.d_cb == 512) return tc::launch_decode_tc_mla(map, a, st);
   switch (hpc_of(c) * 10 + g_of(c)) {
     case 164: return launch_t<4, 16>(map, a, st);
     case 162: return launch_t<2, 16>(map, a, st);

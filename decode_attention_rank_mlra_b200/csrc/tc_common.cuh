@@ -1,0 +1,79 @@
+// Helpers shared by the tensor-core attention kernels (k_decode_tc.cu and
+// k_decode_tc_mla.cu): bounded mbarrier waits, bf16 packing, and the tensor
+// map through which TMA reads the latent cache.
+#pragma once
+
+#include "mlra_internal.cuh"
+#include "sm100_ptx.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace mlra {
+namespace tc {
+
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kBoxCols = 64;             // bf16 columns per TMA box (128 B)
+constexpr int kBoxBytes = kTile * 128;   // 64 rows x 128 B
+constexpr int kSmemLimit = 232448;       // max dynamic shared memory per block
+
+// Bounded mbarrier wait: false on timeout (error recorded) or when another role aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int32_t* err) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer() - t0 > kTimeoutNs) {
+      set_error(err, MLRA_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The cache as a 2-D bf16 tensor [rows, D] (rows = pages * 64, or batch *
+// max_len when contiguous), read in 64 x 64 boxes with the 128-byte swizzle.
+inline cudaError_t make_cache_map(const DecodeArgs& a, CUtensorMap* map) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if (!enc) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  if (!enc) return cudaErrorNotSupported;
+  const mlra_config_t& c = a.cfg;
+  const int D = c.n_blocks * c.d_cb + c.d_r;
+  const uint64_t rows = a.page_table ? uint64_t(a.num_pages) * kPageSize
+                                     : uint64_t(a.batch) * uint64_t(a.max_pages);
+  if (rows >= (uint64_t(1) << 31)) return cudaErrorInvalidValue;
+  cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+  cuuint32_t box[2] = {kBoxCols, kTile};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.kv_cache), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// MLA (one latent block of 512, k_decode_tc_mla.cu): CTAs of 64 heads x one
+// 128-feature quarter of the latent output.
+inline bool mla_supported(const mlra_config_t& c) {
+  return c.n_blocks == 1 && c.d_cb == 512 && c.d_r == 64 && c.n_heads % 64 == 0;
+}
+inline int mla_groups(const mlra_config_t& c) { return (c.n_heads / 64) * 4; }
+cudaError_t launch_decode_tc_mla(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st);
+
+}  // namespace tc
+}  // namespace mlra

@@ -138,6 +138,20 @@ def test_scores_rising_far_above_the_first_tile():
     compare_batch(inp, got)
 
 
+def test_mla_scores_rising_far_above_the_first_tile():
+    """The same rescale path in the MLA kernel (one 512-wide latent block)."""
+    inp = _small("mla_bf16_b8_h128_l131072_paged", 2, [700, 200])
+    flat = inp.kv_cache.view(-1, inp.spec.D)
+    pt = inp.page_table.cpu()
+    for s, first_page in ((0, 1), (1, 2)):
+        for pg in range(first_page, (int(inp.seqlens[s]) + 63) // 64):
+            r0 = int(pt[s, pg]) * 64
+            flat[r0: r0 + 64] *= 3000.0
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    compare_batch(inp, got, heads=[0, 1, 64, 127])
+
+
 def test_scores_falling_far_below_the_first_tile():
     """The first tile holds the largest scores by far: later weights underflow."""
     inp = _small("mlra4_bf16_b64_h32_l16384_paged", 2, [300, 129])
