@@ -36,6 +36,7 @@ using tc::kBoxCols;
 using tc::kSmemLimit;
 using tc::pack_bf16;
 using tc::wait_bar;
+using tc::wait_bar_warp;
 
 constexpr int kThreadsTC = 192;              // warps 0-3 softmax, 4 TMA, 5 MMA
 constexpr uint32_t kTmemCols = 512;
@@ -184,7 +185,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop; each MMA / commit is issued by one elected
     // lane with warp-uniform operands (compile-time offsets from per-stage
-    // descriptors), which keeps the issue rate at the tensor core's pace.
+    // descriptors), which keeps the issue rate at the tensor core's pace.  The
+    // lanes stay converged (the only divergent loop ends in __syncwarp), so
+    // they poll each barrier together and leave a wait together.
     //  QK : S[rows, tokens] = Q[rows, K] . C[tokens, K]^T  (A: TMEM, B: smem K-major)
     //  PV : O[rows, features] += P[rows, tokens] . C_b[tokens, features]
     //       (A: probabilities in TMEM over the S buffer, B: the same tile, MN-major)
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       float m = -INFINITY, l = 0.f;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int sb = it & 1;
-        if (!wait_bar(SFULL(sb), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!wait_bar_warp(SFULL(sb), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         float raw[32];
         {
@@ -435,13 +438,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (__any_sync(0xffffffffu, !(ls <= 0x1p64f))) {
           // rare: a score far above m (or a NaN).  Raise m to this tile's max,
           // rescale l and the O rows once the previous PV is done, redo the tile.
+          // The TMEM pass is taken by the whole warp (alpha = 1 for rows whose
+          // m stays): its loads and stores are warp-wide instructions.
           const float mt = tile_max();
+          float alpha = 1.f;
           if (mt > m) {
-            const float alpha = ex2_approx(m - mt);
+            alpha = ex2_approx(m - mt);
             m = mt;
             l *= alpha;
+          }
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
             const int pk = it - 1;
-            if (!wait_bar(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
+            if (!wait_bar_warp(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
@@ -471,7 +479,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // ---- epilogue: o = (O_hi + O_lo) / l, lse
       {
         const int pk = it - 1;
-        if (!wait_bar(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!wait_bar_warp(PVDONE(pk & 1), (pk >> 1) & 1, abort_flag, err)) { ok = false; break; }
       }
       tc_fence_after();
       const float l_tot = l + __shfl_xor_sync(0xffffffffu, l, 16);

@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
+    // (converged lanes poll each barrier together, as in k_decode_tc.cu)
     constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kTile, false, false);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
     const uint32_t sbase0 = smem_addr(stages);
@@ -295,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // max, moved only when a later tile would overflow (as in k_decode_tc.cu)
       float m = -INFINITY, l = 0.f;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
-        if (!wait_bar(SFULL, it & 1, abort_flag, err)) { ok = false; break; }
+        if (!wait_bar_warp(SFULL, it & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         float raw[32];
         {
@@ -344,25 +345,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__any_sync(0xffffffffu, !(ls <= 0x1p64f))) {
           // rare: a score far above m (or a NaN): raise m, rescale l and the O
           // rows (the previous PV is complete: S of this tile was issued after it)
+          // (the TMEM pass is warp-wide: alpha = 1 for rows whose m stays)
           const float mt = tile_max();
+          float alpha = 1.f;
           if (mt > m) {
-            const float alpha = ex2_approx(m - mt);
+            alpha = ex2_approx(m - mt);
             m = mt;
             l *= alpha;
-            if (t > p.t0) {
-              if (!wait_bar(PVDONE, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
-              tc_fence_after();
+          }
+          if (t > p.t0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            if (!wait_bar_warp(PVDONE, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll 1
-              for (int ch = 0; ch < 4; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(row_t + kColO + 32 * ch, r);
-                tmem_wait_ld();
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t r[32];
+              tmem_ld32(row_t + kColO + 32 * ch, r);
+              tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-                tmem_st32(row_t + kColO + 32 * ch, r);
-              }
-              tmem_wait_st();
+              for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+              tmem_st32(row_t + kColO + 32 * ch, r);
             }
+            tmem_wait_st();
           }
           exps();
         }
@@ -379,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue: o = (O_hi + O_lo) / l for the quarter, lse
-      if (!wait_bar(PVDONE, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
+      if (!wait_bar_warp(PVDONE, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
       const float l_tot = l + __shfl_xor_sync(0xffffffffu, l, 16);
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;

@@ -34,6 +34,15 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// The same wait for a warp whose lanes go on to .sync.aligned instructions
+// (TMEM loads and stores): every lane gets the same answer, so on a timeout
+// the whole warp leaves together instead of a part of it issuing them.
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag, int32_t* err) {
+  const bool good = wait_bar(bar, parity, abort_flag, err);
+  return __all_sync(0xffffffffu, good);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
   return *reinterpret_cast<uint32_t*>(&v);

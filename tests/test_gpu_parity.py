@@ -138,18 +138,36 @@ def test_scores_rising_far_above_the_first_tile():
     compare_batch(inp, got)
 
 
-def test_mla_scores_rising_far_above_the_first_tile():
-    """The same rescale path in the MLA kernel (one 512-wide latent block)."""
-    inp = _small("mla_bf16_b8_h128_l131072_paged", 2, [700, 200])
+def _boost_tokens(inp, seq, first_token, factor):
+    """Multiply the cache rows of tokens >= first_token of one sequence."""
+    L = int(inp.seqlens[seq])
+    if inp.page_table is None:
+        inp.kv_cache[seq, first_token:L] *= factor
+        return
     flat = inp.kv_cache.view(-1, inp.spec.D)
     pt = inp.page_table.cpu()
-    for s, first_page in ((0, 1), (1, 2)):
-        for pg in range(first_page, (int(inp.seqlens[s]) + 63) // 64):
-            r0 = int(pt[s, pg]) * 64
-            flat[r0: r0 + 64] *= 3000.0
+    for t0 in range(first_token, L, 64):
+        r0 = int(pt[seq, t0 // 64]) * 64
+        flat[r0 + t0 % 64: r0 + 64] *= factor
+
+
+@pytest.mark.parametrize("name,factor", [
+    ("mla_bf16_b8_h128_l131072_paged", 3000.0),
+    ("mla_bf16_b8_h128_l131072_paged", 20.0),
+    ("mlra4_bf16_b64_h32_l16384_paged", 20.0),
+    ("mlra4_bf16_b128_h16_ragged1k_64k_paged", 20.0),
+])
+def test_scores_rising_in_some_heads_only(name, factor):
+    """Later tiles overflow the first tile's reference point in all heads
+    (x3000) or only in some heads of a warp (x20): the rescale of O is taken
+    by whole warps either way.  Pieces span several tiles."""
+    inp = _small(name, 2, [3000, 2000])
+    _boost_tokens(inp, 0, 200, factor)
+    _boost_tokens(inp, 1, 1000, factor)
     got = run_gpu(inp)
     assert got["device_error"] == 0
-    compare_batch(inp, got, heads=[0, 1, 64, 127])
+    heads = sorted({0, 1, inp.spec.n_heads // 2 + 1, inp.spec.n_heads - 1})
+    compare_batch(inp, got, heads=heads)
 
 
 def test_scores_falling_far_below_the_first_tile():
