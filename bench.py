@@ -209,7 +209,7 @@ def measured_traffic(workload: str):
             t = json.load(f)
         h = hashlib.sha256()
         csrc = os.path.join(ROOT, "decode_attention_rank_mlra_b200", "csrc")
-        for name in ("k_decode_tc.cu", "sm100_ptx.cuh", "mlra_internal.cuh"):
+        for name in t["sources"]:
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(f.read())
         if h.hexdigest() != t["sources_sha256"]:
