@@ -45,3 +45,9 @@ from .mlra_oracle import (  # noqa: F401
     decode_sampled,
     SeqResult,
 )
+from .cache_oracle import (  # noqa: F401
+    kv_scale,
+    rms_norm_blocks,
+    rope,
+    cache_rows,
+)

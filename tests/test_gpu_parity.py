@@ -80,6 +80,23 @@ def test_batches_spanning_several_sequence_tiles(batch, fused):
     compare_batch(inp, got, seqs=pick, heads=[0, 13, 31])
 
 
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("heads", [16, 32, 64])
+def test_mlra2_two_branches(heads, fused):
+    """MLRA-2 (two latent blocks of 128, branch rescale 1/sqrt(2)): the same
+    kernels with two branches per CTA (h <= 32) or one (h = 64)."""
+    base = W.WORKLOADS["mlra4_bf16_b64_h32_l16384_paged"]
+    seqlens = [1, 64, 700, 1300, 333]
+    spec = W.scaled_down(base, len(seqlens), seqlen=max(seqlens), n_heads=heads, seed=23)
+    spec = spec.replace(n_blocks=2, name=spec.name + "_mlra2")
+    assert spec.D == 320 and abs(spec.branch_scale - 2 ** -0.5) < 1e-12
+    inp = W.make_inputs(spec, "cuda", seqlens=np.asarray(seqlens, np.int32))
+    got = run_gpu(inp, fused=fused)
+    assert got["device_error"] == 0
+    assert mlra.decode_kernel_kind(config_of(spec)) == "tcgen05"
+    compare_batch(inp, got, heads=sorted({0, heads // 2, heads - 1}))
+
+
 def test_fused_projection_without_latent_outputs():
     """combine_out_proj with o_latent = lse = None gives the same out."""
     inp = _small("mlra4_bf16_b16_h16_l4096_contig", 3, [500, 64, 1])

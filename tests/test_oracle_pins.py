@@ -214,7 +214,7 @@ def test_shift_invariance_through_rope():
                                rtol=1e-10, atol=1e-12)
 
 
-@pytest.mark.parametrize("nb", [1, 4])
+@pytest.mark.parametrize("nb", [1, 2, 4])
 def test_absorbed_equals_unabsorbed(nb):
     """Main Findings: decoding reduces to absorbable steps, so the absorbed form
     (query absorption, attention over the latent, output up-projection) gives
