@@ -336,7 +336,17 @@ def run_ours(args):
                                                   dec.workspace),
         "combine_out_proj": lambda i: mlra.combine_out_proj(cfg, dec.workspace, B, inp.w_uv,
                                                             dec.out, dec.o_latent, dec.lse),
+        # the cache-write step (not part of the step above): every sequence's
+        # last row rewritten from a normalised latent and a rotated RoPE key
+        "cache_append": lambda i: mlra.cache_append(cfg, app_c, app_kr, app_gamma, 2.0,
+                                                    caches[i % copies], inp.page_table, app_pos,
+                                                    max_pages),
     }
+    g_app = torch.Generator().manual_seed(1)
+    app_c = torch.randn(B, spec.n_blocks * spec.d_cb, generator=g_app).to(spec.torch_dtype).to(dev)
+    app_kr = torch.randn(B, spec.d_r, generator=g_app).to(spec.torch_dtype).to(dev)
+    app_gamma = torch.ones(spec.n_blocks * spec.d_cb, dtype=torch.float32, device=dev)
+    app_pos = (inp.seqlens - 1).clamp(min=0)
     breakdown = {}
     n_rep = 2 * copies
     for name, fn in calls.items():

@@ -38,6 +38,7 @@ EXPORTS = [
     "mlra_status_string", "mlra_version", "mlra_absorb_q", "mlra_workspace_size",
     "mlra_decode_attn", "mlra_splitkv_combine", "mlra_out_proj", "mlra_get_device_error",
     "mlra_decode_kernel_kind", "mlra_decode_attn_noalloc", "mlra_combine_out_proj",
+    "mlra_cache_append",
 ]
 
 
@@ -100,6 +101,8 @@ def lib() -> ctypes.CDLL:
         "mlra_splitkv_combine": (I32, [CP, P, SZ, I32, P, P, P]),
         "mlra_out_proj": (I32, [CP, P, P, P, I32, P]),
         "mlra_combine_out_proj": (I32, [CP, P, SZ, I32, P, P, P, P, P]),
+        "mlra_cache_append": (I32, [CP, P, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_float, P,
+                                    I64, P, I32, P, I32, P, P]),
         "mlra_get_device_error": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "mlra_decode_kernel_kind": (I32, [CP]),
         "mlra_decode_attn_noalloc": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, P, P, P]),
@@ -248,6 +251,31 @@ def combine_out_proj(cfg: Config, workspace: torch.Tensor, batch: int, w_uv: tor
     return out
 
 
+def cache_append(cfg: Config, c_new: torch.Tensor, k_rope_new: torch.Tensor,
+                 rms_gamma: torch.Tensor, alpha_kv: float, kv_cache: torch.Tensor,
+                 page_table: Optional[torch.Tensor], positions: torch.Tensor, max_pages: int,
+                 rms_eps: float = 1e-6, rope_theta: float = 10000.0,
+                 device_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Cache write: each sequence's new row (per-block RMSNorm x gain x alpha_kv,
+    rotated RoPE key) at token ``positions[s]``, in place in ``kv_cache``."""
+    _need(c_new, "c_new", cfg.torch_dtype)
+    _need(k_rope_new, "k_rope_new", cfg.torch_dtype)
+    _need(rms_gamma, "rms_gamma", torch.float32)
+    _need(kv_cache, "kv_cache", cfg.torch_dtype)
+    _need(positions, "positions", torch.int32)
+    num_pages = 0
+    if page_table is not None:
+        _need(page_table, "page_table", torch.int32)
+        num_pages = kv_cache.shape[0]
+    if device_status is not None:
+        _need(device_status, "device_status", torch.int32)
+    B = positions.shape[0]
+    _check("mlra_cache_append", lib().mlra_cache_append(
+        ctypes.byref(cfg), _ptr(c_new), _ptr(k_rope_new), _ptr(rms_gamma), float(alpha_kv),
+        float(rms_eps), float(rope_theta), _ptr(kv_cache), num_pages, _ptr(page_table),
+        int(max_pages), _ptr(positions), B, _ptr(device_status), _stream(stream)))
+
+
 def decode_attn_noalloc(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor,
                         kv_cache: torch.Tensor, page_table: Optional[torch.Tensor],
                         seqlens: torch.Tensor, max_pages: int, o_latent: torch.Tensor,
@@ -334,7 +362,8 @@ class Decoder:
 
 __all__ = [
     "Config", "make_config", "lib", "absorb_q", "workspace_size", "alloc_workspace",
-    "decode_attn", "splitkv_combine", "out_proj", "combine_out_proj", "get_device_error",
+    "decode_attn", "splitkv_combine", "out_proj", "combine_out_proj", "cache_append",
+    "get_device_error",
     "decode_kernel_kind", "decode_attn_noalloc",
     "Decoder", "MlraError", "EXPORTS", "F32", "BF16",
 ]

@@ -266,6 +266,36 @@ mlra_status_t mlra_combine_out_proj(const mlra_config_t* cfg, const void* worksp
   return from_cuda(launch_out_proj(*cfg, o_latent, w_uv, out, batch, s));
 }
 
+mlra_status_t mlra_cache_append(const mlra_config_t* cfg, const void* c_new,
+                                const void* k_rope_new, const float* rms_gamma, float alpha_kv,
+                                float rms_eps, float rope_theta, void* kv_cache,
+                                int64_t num_pages, const int32_t* page_table, int32_t max_pages,
+                                const int32_t* positions, int32_t batch, int32_t* device_status,
+                                mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0) return MLRA_ERR_INVALID_ARG;
+  if (batch == 0) return MLRA_OK;
+  if (!c_new || !k_rope_new || !rms_gamma || !kv_cache || !positions) return MLRA_ERR_INVALID_ARG;
+  if (cfg->d_r % 2 != 0 || max_pages < 1) return MLRA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !(rms_eps >= 0.f) || !(alpha_kv == alpha_kv)) return MLRA_ERR_INVALID_ARG;
+  if (page_table) {
+    if (cfg->page_size != kPageSize) return MLRA_ERR_UNSUPPORTED;
+    if (num_pages < 1 || num_pages > (int64_t(1) << 31) / kPageSize) return MLRA_ERR_INVALID_ARG;
+  }
+  const uintptr_t el = cfg->dtype == MLRA_BF16 ? 2 : 4;
+  if (!aligned(c_new, el) || !aligned(k_rope_new, el) || !aligned(kv_cache, el) ||
+      !aligned(rms_gamma, 4) || !aligned(positions, 4) || (page_table && !aligned(page_table, 4)) ||
+      (device_status && !aligned(device_status, 4)))
+    return MLRA_ERR_ALIGNMENT;
+  const int64_t cap64 = page_table ? int64_t(max_pages) * kPageSize : int64_t(max_pages);
+  if (cap64 > (int64_t(1) << 30)) return MLRA_ERR_INVALID_ARG;
+  return from_cuda(launch_cache_append(*cfg, c_new, k_rope_new, rms_gamma, alpha_kv, rms_eps,
+                                       double(rope_theta), kv_cache, page_table ? num_pages : 0,
+                                       page_table, max_pages, int(cap64), positions, batch,
+                                       device_status, (cudaStream_t)stream));
+}
+
 mlra_status_t mlra_get_device_error(const void* workspace, size_t workspace_bytes,
                                     int32_t* device_status, mlra_stream_t stream) {
   if (!workspace || !device_status || workspace_bytes < sizeof(WsHeader))

@@ -279,6 +279,13 @@ struct DecodeArgs {
   int32_t n_groups;
 };
 
+// Cache write (k_cache.cu).
+cudaError_t launch_cache_append(const mlra_config_t& c, const void* c_new, const void* k_rope_new,
+                                const float* gamma, float alpha_kv, float eps, double theta,
+                                void* kv_cache, int64_t num_pages, const int32_t* page_table,
+                                int max_pages, int cap, const int32_t* positions, int batch,
+                                int32_t* status, cudaStream_t st);
+
 // Tensor-core absorption and output projection (bf16, d_h = 128).
 bool proj_tc_supported(const mlra_config_t& c);
 cudaError_t launch_absorb_tc(const mlra_config_t& c, const void* q_nope, const void* w_uk,

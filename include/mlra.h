@@ -190,6 +190,35 @@ MLRA_API mlra_status_t mlra_combine_out_proj(const mlra_config_t* cfg, const voi
                                     mlra_stream_t stream);
 
 /*
+ * Cache write (the step before decode attention reads the cache; the paper
+ * describes it in prose: Methodology, third paragraph, latent RMSNorm before
+ * the up-projection; Main Findings, variance bullet, the KV latent scaled by
+ * alpha_kv; Key Contributions #2, one decoupled RoPE key).  For every
+ * sequence s, the row of its new token at position p = positions[s]:
+ *   latent block b: alpha_kv * gamma * c_b / sqrt(mean(c_b^2) + rms_eps)
+ *   RoPE key: channel i paired with i + d_r/2, rotated by p * theta^(-2i/d_r)
+ *   c_new      : [batch, n_blocks * d_cb] dtype (latent before normalisation)
+ *   k_rope_new : [batch, d_r] dtype (RoPE key before rotation; d_r even)
+ *   rms_gamma  : [n_blocks * d_cb] fp32 gain
+ *   alpha_kv   : the latent scale (sqrt(d_model / d_cb) in the paper's calibration)
+ *   kv_cache, num_pages, page_table, max_pages : as mlra_decode_attn; the row
+ *                of token p is written in place (page_table[s][p / 64], row p % 64)
+ *   positions  : [batch] int32, 0 <= p < max_pages * 64 (paged) or < max_len
+ *   device_status : one int32 in device memory or NULL; a position out of
+ *                range (MLRA_ERR_INVALID_ARG) or a page id out of range
+ *                (MLRA_ERR_BAD_PAGE) is recorded there (first error wins) and
+ *                that sequence's row is not written.
+ * Pointers must be aligned to their element type.  No counterpart to the
+ * paper's kernels: it fixes no layout for this step.
+ */
+MLRA_API mlra_status_t mlra_cache_append(const mlra_config_t* cfg, const void* c_new,
+                                const void* k_rope_new, const float* rms_gamma, float alpha_kv,
+                                float rms_eps, float rope_theta, void* kv_cache,
+                                int64_t num_pages, const int32_t* page_table, int32_t max_pages,
+                                const int32_t* positions, int32_t batch, int32_t* device_status,
+                                mlra_stream_t stream);
+
+/*
  * Read (and then clear) the device error word of a workspace.  Synchronises
  * `stream`.  *device_status receives MLRA_OK or the first device-side error
  * (MLRA_ERR_BAD_PAGE, MLRA_ERR_TIMEOUT) recorded since the last decode call.
