@@ -12,7 +12,7 @@ LIB = os.path.join(HERE, "libmlra.so")
 SOURCES = ["mlra_api.cu", "k_small.cu", "k_decode_simt.cu", "k_decode_tc.cu", "k_decode_tc_mla.cu",
            "k_proj_tc.cu", "k_cache.cu",
            "k_noalloc.cu"]
-HEADERS = ["mlra_internal.cuh", "sm100_ptx.cuh", "../../include/mlra.h"]
+HEADERS = ["mlra_internal.cuh", "dispatch.h", "tc_common.cuh", "sm100_ptx.cuh", "../../include/mlra.h"]
 
 
 def nvcc_path() -> str:

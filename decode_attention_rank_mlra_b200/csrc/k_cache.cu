@@ -15,7 +15,7 @@
 // warp at a time), warp 4 rotates the RoPE key.  The rotation angle and its
 // sine and cosine are taken in fp64: at positions near 2^17 an fp32 angle is
 // off by ~1e-2 rad.
-#include "mlra_internal.cuh"
+#include "dispatch.h"
 
 #include <math.h>
 

@@ -10,7 +10,7 @@
 // CTA work: group g = (head group of 16, branch b); the CTA walks its share of
 // the tile stream, in sub-tiles of 32 tokens staged in shared memory as fp32.
 // 128 threads: head slot i = tid / 8, sub = tid % 8.
-#include "mlra_internal.cuh"
+#include "dispatch.h"
 
 #include <math.h>
 

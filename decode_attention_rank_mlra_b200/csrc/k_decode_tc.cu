@@ -23,6 +23,7 @@
 // Precision: queries and probabilities are carried as bf16 hi + lo pairs (two
 // MMA rows per head), so both enter the fp32-accumulated products with about
 // 16 significant bits while the cache stays the bf16 it is stored as.
+#include "dispatch.h"
 #include "tc_common.cuh"
 
 #include <math.h>

@@ -14,7 +14,7 @@
 //  * out_proj: D[j, s] = sum_k W_uv[k, j] o[s, k]        (A = W_uv MN-major,
 //             B = o as bf16 hi + lo pairs written by the CTA's threads, so the
 //             fp32 o enters with ~16 significant bits).
-#include "mlra_internal.cuh"
+#include "dispatch.h"
 #include "sm100_ptx.cuh"
 
 #include <cudaTypedefs.h>

@@ -2,7 +2,7 @@
 // combine and output up-projection.  All fp32 SIMT: together they move well
 // under 5% of the bytes of the attention kernel (see the layer description in
 // include/mlra.h for the maths).
-#include "mlra_internal.cuh"
+#include "dispatch.h"
 
 #include <math.h>
 

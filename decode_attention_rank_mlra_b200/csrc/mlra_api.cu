@@ -1,7 +1,7 @@
 // Host side of the C ABI declared in include/mlra.h: argument validation,
 // workspace layout, kernel selection and launches.  No allocation, no host
 // synchronisation (except mlra_get_device_error).
-#include "mlra_internal.cuh"
+#include "dispatch.h"
 
 #include <stdlib.h>
 #include <string.h>
