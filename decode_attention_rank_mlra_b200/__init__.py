@@ -38,7 +38,7 @@ EXPORTS = [
     "mlra_status_string", "mlra_version", "mlra_absorb_q", "mlra_workspace_size",
     "mlra_decode_attn", "mlra_splitkv_combine", "mlra_out_proj", "mlra_get_device_error",
     "mlra_decode_kernel_kind", "mlra_decode_attn_noalloc", "mlra_combine_out_proj",
-    "mlra_cache_append",
+    "mlra_cache_append", "mlra_step_workspace_size", "mlra_decode_step",
 ]
 
 
@@ -106,6 +106,8 @@ def lib() -> ctypes.CDLL:
         "mlra_get_device_error": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "mlra_decode_kernel_kind": (I32, [CP]),
         "mlra_decode_attn_noalloc": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, P, P, P]),
+        "mlra_step_workspace_size": (I32, [CP, I32, ctypes.POINTER(SZ)]),
+        "mlra_decode_step": (I32, [CP, P, P, P, I32, P, P, P, I64, P, I32, P, I32, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -120,13 +122,19 @@ def status_string(status: int) -> str:
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
-def _stream(stream) -> ctypes.c_void_p:
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream) -> int:
+    """cudaStream_t of ``stream`` (default: the current stream of the current device)."""
     if stream is None:
+        if _raw_stream is not None:
+            return _raw_stream(torch._C._cuda_getDevice())
         stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    return stream.cuda_stream
 
 
 def _need(t: torch.Tensor, name: str, dtype: Optional[torch.dtype] = None):
@@ -166,11 +174,8 @@ def workspace_size(cfg: Config, batch: int) -> int:
 
 
 def alloc_workspace(cfg: Config, batch: int, device=None) -> torch.Tensor:
-    """Caller-owned workspace (uint8, 256-byte aligned by the caching allocator)."""
-    n = workspace_size(cfg, batch)
-    ws = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
-    off = (-ws.data_ptr()) % 256
-    return ws[off: off + n]
+    """Caller-owned workspace (uint8, 256-byte aligned)."""
+    return _aligned_bytes(workspace_size(cfg, batch), device)
 
 
 def decode_attn(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor, kv_cache: torch.Tensor,
@@ -276,6 +281,69 @@ def cache_append(cfg: Config, c_new: torch.Tensor, k_rope_new: torch.Tensor,
         int(max_pages), _ptr(positions), B, _ptr(device_status), _stream(stream)))
 
 
+def step_workspace_size(cfg: Config, batch: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mlra_step_workspace_size", lib().mlra_step_workspace_size(ctypes.byref(cfg), batch,
+                                                                      ctypes.byref(n)))
+    return int(n.value)
+
+
+def _aligned_bytes(n: int, device) -> torch.Tensor:
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
+    off = (-ws.data_ptr()) % 256
+    return ws[off: off + n]
+
+
+def alloc_step_workspace(cfg: Config, batch: int, device=None) -> torch.Tensor:
+    """Caller-owned workspace for ``decode_step`` (its first
+    ``workspace_size`` bytes serve as the decode workspace)."""
+    return _aligned_bytes(step_workspace_size(cfg, batch), device)
+
+
+def decode_step(cfg: Config, q_nope: torch.Tensor, q_rope: torch.Tensor, seqlens: torch.Tensor,
+                w_uk: torch.Tensor, w_uv: torch.Tensor, kv_cache: torch.Tensor,
+                page_table: Optional[torch.Tensor], max_pages: int, out: torch.Tensor,
+                workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """Steps 1, 2a, 2b and 3 in one library call (absorb, attention, merge,
+    output projection), bitwise equal to the three separate calls.
+
+    ``q_nope``, ``q_rope``, ``seqlens`` and ``out`` are either all CUDA
+    tensors or all host tensors (page-locked for an asynchronous call).  With
+    host tensors the library moves them on ``stream`` (page-locked memory by
+    one staging kernel and in-place output stores, other memory by copies);
+    ``out`` is valid once the stream has passed the call.
+    """
+    on_host = not q_nope.is_cuda
+    if q_rope.is_cuda == on_host or seqlens.is_cuda == on_host or out.is_cuda == on_host:
+        raise ValueError("q_nope, q_rope, seqlens and out must all be on the host "
+                         "or all on the device")
+    if not (q_nope.is_contiguous() and q_rope.is_contiguous() and seqlens.is_contiguous()
+            and out.is_contiguous()):
+        raise ValueError("q_nope, q_rope, seqlens and out must be contiguous")
+    dt = cfg.torch_dtype
+    if q_nope.dtype != dt or q_rope.dtype != dt or seqlens.dtype != torch.int32 \
+            or out.dtype != torch.float32:
+        raise ValueError(f"dtypes must be q_nope/q_rope {dt}, seqlens int32, out float32")
+    B = seqlens.shape[0]
+    h = cfg.n_heads
+    if q_nope.shape != (B, h, cfg.d_h) or q_rope.shape != (B, h, cfg.d_r) \
+            or out.shape != (B, h, cfg.d_h):
+        raise ValueError("q_nope / q_rope / out shapes do not match seqlens and cfg")
+    _need(w_uk, "w_uk", cfg.torch_dtype)
+    _need(w_uv, "w_uv", cfg.torch_dtype)
+    _need(kv_cache, "kv_cache", cfg.torch_dtype)
+    _need(workspace, "workspace", torch.uint8)
+    num_pages = 0
+    if page_table is not None:
+        _need(page_table, "page_table", torch.int32)
+        num_pages = kv_cache.shape[0]
+    _check("mlra_decode_step", lib().mlra_decode_step(
+        ctypes.byref(cfg), _ptr(q_nope), _ptr(q_rope), _ptr(seqlens), B, _ptr(w_uk), _ptr(w_uv),
+        _ptr(kv_cache), num_pages, _ptr(page_table), int(max_pages), _ptr(out), int(on_host),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
 def decode_attn_noalloc(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor,
                         kv_cache: torch.Tensor, page_table: Optional[torch.Tensor],
                         seqlens: torch.Tensor, max_pages: int, o_latent: torch.Tensor,
@@ -330,7 +398,9 @@ class Decoder:
 
     ``run`` launches absorb -> decode_attn -> splitkv_combine -> out_proj on
     the current stream and returns ``out`` [B, h, d_h] fp32; with
-    ``fused=True`` the last two are one combine_out_proj call.
+    ``fused=True`` the last two are one combine_out_proj call.  ``step`` makes
+    the same computation one library call (``decode_step``), from device or
+    host buffers.
     """
 
     cfg: Config
@@ -339,7 +409,8 @@ class Decoder:
 
     def __post_init__(self):
         c, B, dev = self.cfg, self.batch, self.device
-        self.workspace = alloc_workspace(c, B, dev)
+        self.step_workspace = alloc_step_workspace(c, B, dev)
+        self.workspace = self.step_workspace[: workspace_size(c, B)]
         self.q_abs = torch.empty((B, c.n_heads, c.n_blocks, c.d_cb), dtype=torch.float32, device=dev)
         self.o_latent = torch.empty((B, c.n_heads, c.n_blocks, c.d_cb), dtype=torch.float32,
                                     device=dev)
@@ -359,11 +430,19 @@ class Decoder:
             out_proj(self.cfg, self.o_latent, w_uv, self.out, stream)
         return self.out
 
+    def step(self, q_nope, q_rope, seqlens, w_uk, w_uv, kv_cache, page_table, max_pages,
+             out=None, stream=None) -> torch.Tensor:
+        if out is None:
+            out = self.out
+        return decode_step(self.cfg, q_nope, q_rope, seqlens, w_uk, w_uv, kv_cache, page_table,
+                           max_pages, out, self.step_workspace, stream)
+
 
 __all__ = [
     "Config", "make_config", "lib", "absorb_q", "workspace_size", "alloc_workspace",
     "decode_attn", "splitkv_combine", "out_proj", "combine_out_proj", "cache_append",
     "get_device_error",
-    "decode_kernel_kind", "decode_attn_noalloc",
+    "decode_kernel_kind", "decode_attn_noalloc", "step_workspace_size", "alloc_step_workspace",
+    "decode_step",
     "Decoder", "MlraError", "EXPORTS", "F32", "BF16",
 ]

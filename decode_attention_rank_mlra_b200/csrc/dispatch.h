@@ -16,6 +16,15 @@ cudaError_t launch_combine(const mlra_config_t& c, const void* ws, const WsLayou
 cudaError_t launch_out_proj(const mlra_config_t& c, const float* o_latent, const void* w_uv,
                             float* out, int batch, cudaStream_t st);
 
+// Copies of up to three byte ranges in one launch, each source being host
+// memory mapped into the device address space (k_small.cu).
+struct StageCopy {
+  const void* src;
+  void* dst;
+  size_t bytes;
+};
+cudaError_t launch_stage(const StageCopy* copies, int n, cudaStream_t st);
+
 // Cache write (k_cache.cu).
 cudaError_t launch_cache_append(const mlra_config_t& c, const void* c_new, const void* k_rope_new,
                                 const float* gamma, float alpha_kv, float eps, double theta,

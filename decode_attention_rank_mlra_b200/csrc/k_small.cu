@@ -6,6 +6,8 @@
 
 #include <math.h>
 
+#include <algorithm>
+
 namespace mlra {
 
 template <typename T> __device__ __forceinline__ float ld_f32(const T* p);
@@ -405,6 +407,78 @@ cudaError_t launch_out_proj(const mlra_config_t& c, const float* o_latent, const
   return launch_pdl(out_proj_kernel<float>, grid, dim3(kOpWarps * 32), sm, st, o_latent,
                     (const float*)w_uv, out, batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h,
                     c.branch_scale);
+}
+
+// ---------------------------------------------------------------------------
+// Staging of a step's inputs from page-locked host memory: the kernel reads
+// the mapped host ranges directly (bypassing the cache, the host rewrites them
+// between steps) and writes the workspace.  At decode sizes (tens of KB) one
+// launch costs a PCIe round trip, where each copy-engine transfer carries a
+// fixed cost several times larger.
+namespace {
+
+struct StageArgs {
+  StageCopy c[3];
+  int n;
+};
+
+template <typename U>
+__device__ __forceinline__ void stage_units(const void* src, void* dst, size_t n, size_t tid,
+                                            size_t nth) {
+  const U* s = static_cast<const U*>(src);
+  U* d = static_cast<U*>(dst);
+  size_t i = tid;
+  // four loads in flight per thread before the first store
+  for (; i + 3 * nth < n; i += 4 * nth) {
+    const U v0 = __ldcv(s + i), v1 = __ldcv(s + i + nth), v2 = __ldcv(s + i + 2 * nth),
+            v3 = __ldcv(s + i + 3 * nth);
+    d[i] = v0;
+    d[i + nth] = v1;
+    d[i + 2 * nth] = v2;
+    d[i + 3 * nth] = v3;
+  }
+  for (; i < n; i += nth) d[i] = __ldcv(s + i);
+}
+
+__host__ __device__ inline int stage_unit(const StageCopy& c) {
+  const uintptr_t m = reinterpret_cast<uintptr_t>(c.src) | reinterpret_cast<uintptr_t>(c.dst) |
+                      uintptr_t(c.bytes);
+  return (m & 15) == 0 ? 16 : (m & 7) == 0 ? 8 : (m & 3) == 0 ? 4 : (m & 1) == 0 ? 2 : 1;
+}
+
+__global__ void __launch_bounds__(256) stage_kernel(StageArgs a) {
+  // the previous step's kernels may still read the destination
+  pdl_wait();
+  pdl_trigger();
+  const size_t tid = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t nth = size_t(gridDim.x) * blockDim.x;
+  for (int k = 0; k < a.n; ++k) {
+    const StageCopy& c = a.c[k];
+    switch (stage_unit(c)) {
+      case 16: stage_units<uint4>(c.src, c.dst, c.bytes / 16, tid, nth); break;
+      case 8: stage_units<uint2>(c.src, c.dst, c.bytes / 8, tid, nth); break;
+      case 4: stage_units<unsigned int>(c.src, c.dst, c.bytes / 4, tid, nth); break;
+      case 2: stage_units<unsigned short>(c.src, c.dst, c.bytes / 2, tid, nth); break;
+      default: stage_units<unsigned char>(c.src, c.dst, c.bytes, tid, nth); break;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_stage(const StageCopy* copies, int n, cudaStream_t st) {
+  if (n < 1 || n > 3) return cudaErrorInvalidValue;
+  StageArgs a{};
+  a.n = n;
+  size_t units = 0;
+  for (int k = 0; k < n; ++k) {
+    a.c[k] = copies[k];
+    units = std::max(units, copies[k].bytes / size_t(stage_unit(copies[k])));
+  }
+  // one unit per thread up to 4 waves of 148 CTAs; beyond that each thread
+  // loops, four loads at a time
+  const size_t blocks = std::min<size_t>(std::max<size_t>((units + 255) / 256, 1), 592);
+  return launch_pdl(stage_kernel, dim3(unsigned(blocks)), dim3(256), 0, st, a);
 }
 
 }  // namespace mlra

@@ -99,6 +99,49 @@ WsLayout layout_for(const mlra_config_t& c, int batch, const Grid& g) {
 
 mlra_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
 
+// Device address of the host range [p, p + bytes) when it is page-locked and
+// mapped into the current device's address space (checked at both ends), else
+// NULL, in which case no kernel ever dereferences it.
+const void* mapped_host_range(const void* p, size_t bytes) {
+  if (!p || bytes == 0) return nullptr;
+  cudaPointerAttributes a0{}, a1{};
+  const char* last = static_cast<const char*>(p) + (bytes - 1);
+  if (cudaPointerGetAttributes(&a0, p) != cudaSuccess ||
+      cudaPointerGetAttributes(&a1, last) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (a0.type != cudaMemoryTypeHost || a1.type != cudaMemoryTypeHost || !a0.devicePointer ||
+      !a1.devicePointer)
+    return nullptr;
+  if (static_cast<const char*>(a1.devicePointer) - static_cast<const char*>(a0.devicePointer) !=
+      ptrdiff_t(bytes - 1))
+    return nullptr;
+  return a0.devicePointer;
+}
+
+// mlra_decode_step's workspace: the decode workspace, then its own buffers,
+// each starting on a 256-byte boundary.
+struct StepLayout {
+  size_t attn, q_abs, o_lat, q_nope, q_rope, seqlens, out, total;
+};
+
+StepLayout step_layout(const mlra_config_t& c, int batch, const Grid& g) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t esz = c.dtype == MLRA_BF16 ? 2 : 4;
+  const size_t bh = size_t(batch) * c.n_heads, K = size_t(c.n_blocks) * c.d_cb;
+  StepLayout s;
+  s.attn = up(layout_for(c, batch, g).total);
+  s.q_abs = s.attn;
+  s.o_lat = s.q_abs + up(bh * K * 4);
+  s.q_nope = s.o_lat + up(bh * K * 4);
+  s.q_rope = s.q_nope + up(bh * c.d_h * esz);
+  s.seqlens = s.q_rope + up(bh * c.d_r * esz);
+  s.out = s.seqlens + up(size_t(batch) * 4);
+  s.total = s.out + up(bh * c.d_h * 4);
+  return s;
+}
+
 }  // namespace
 
 extern "C" {
@@ -264,6 +307,87 @@ mlra_status_t mlra_combine_out_proj(const mlra_config_t* cfg, const void* worksp
   cudaError_t e = launch_combine(*cfg, workspace, L, batch, o_latent, lse, s);
   if (e != cudaSuccess) return MLRA_ERR_CUDA;
   return from_cuda(launch_out_proj(*cfg, o_latent, w_uv, out, batch, s));
+}
+
+mlra_status_t mlra_step_workspace_size(const mlra_config_t* cfg, int32_t batch, size_t* bytes) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0 || !bytes) return MLRA_ERR_INVALID_ARG;
+  Grid g;
+  st = plan_grid(*cfg, &g);
+  if (st != MLRA_OK) return st;
+  *bytes = step_layout(*cfg, batch, g).total;
+  return MLRA_OK;
+}
+
+mlra_status_t mlra_decode_step(const mlra_config_t* cfg, const void* q_nope, const void* q_rope,
+                               const int32_t* seqlens, int32_t batch, const void* w_uk,
+                               const void* w_uv, const void* kv_cache, int64_t num_pages,
+                               const int32_t* page_table, int32_t max_pages, float* out,
+                               int32_t host_io, void* workspace, size_t workspace_bytes,
+                               mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0 || !workspace || (host_io != 0 && host_io != 1)) return MLRA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLRA_ERR_WORKSPACE;
+  if (batch == 0) return MLRA_OK;
+  if (!q_nope || !q_rope || !seqlens || !w_uk || !w_uv || !kv_cache || !out)
+    return MLRA_ERR_INVALID_ARG;
+  Grid g;
+  st = plan_grid(*cfg, &g);
+  if (st != MLRA_OK) return st;
+  const StepLayout S = step_layout(*cfg, batch, g);
+  if (workspace_bytes < S.total) return MLRA_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t esz = cfg->dtype == MLRA_BF16 ? 2 : 4;
+  const size_t bh = size_t(batch) * cfg->n_heads;
+  float* dev_out = out;
+  bool copy_out = false;
+  if (host_io) {
+    // Inputs: ranges the device can read in place move in one staging launch,
+    // any others (pageable memory) by copy-engine transfers.
+    const void* src[3] = {q_nope, q_rope, seqlens};
+    const size_t off[3] = {S.q_nope, S.q_rope, S.seqlens};
+    const size_t len[3] = {bh * cfg->d_h * esz, bh * cfg->d_r * esz, size_t(batch) * 4};
+    StageCopy staged[3];
+    int n_staged = 0;
+    for (int k = 0; k < 3; ++k) {
+      if (const void* d = mapped_host_range(src[k], len[k])) {
+        staged[n_staged++] = StageCopy{d, ws + off[k], len[k]};
+      } else if (cudaMemcpyAsync(ws + off[k], src[k], len[k], cudaMemcpyHostToDevice, s) !=
+                 cudaSuccess) {
+        return MLRA_ERR_CUDA;
+      }
+    }
+    if (n_staged > 0 && launch_stage(staged, n_staged, s) != cudaSuccess) return MLRA_ERR_CUDA;
+    q_nope = ws + S.q_nope;
+    q_rope = ws + S.q_rope;
+    seqlens = reinterpret_cast<const int32_t*>(ws + S.seqlens);
+    // Output: written by the projection kernel straight into mapped host
+    // memory, else into the workspace and copied back.
+    if (void* d = const_cast<void*>(mapped_host_range(out, bh * cfg->d_h * 4))) {
+      dev_out = static_cast<float*>(d);
+    } else {
+      dev_out = reinterpret_cast<float*>(ws + S.out);
+      copy_out = true;
+    }
+  }
+  float* q_abs = reinterpret_cast<float*>(ws + S.q_abs);
+  st = mlra_absorb_q(cfg, q_nope, w_uk, q_abs, batch, stream);
+  if (st != MLRA_OK) return st;
+  st = mlra_decode_attn(cfg, q_abs, q_rope, kv_cache, num_pages, page_table, max_pages, seqlens,
+                        batch, workspace, S.attn, stream);
+  if (st != MLRA_OK) return st;
+  // The fused kernel needs no latent output; where it does not apply, the
+  // two-kernel fallback writes it to the workspace.
+  st = mlra_combine_out_proj(cfg, workspace, S.attn, batch, w_uv, dev_out, nullptr, nullptr,
+                             stream);
+  if (st == MLRA_ERR_UNSUPPORTED)
+    st = mlra_combine_out_proj(cfg, workspace, S.attn, batch, w_uv, dev_out,
+                               reinterpret_cast<float*>(ws + S.o_lat), nullptr, stream);
+  if (st != MLRA_OK || !copy_out) return st;
+  return from_cuda(cudaMemcpyAsync(out, dev_out, bh * cfg->d_h * 4, cudaMemcpyDeviceToHost, s));
 }
 
 mlra_status_t mlra_cache_append(const mlra_config_t* cfg, const void* c_new,

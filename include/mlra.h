@@ -190,6 +190,47 @@ MLRA_API mlra_status_t mlra_combine_out_proj(const mlra_config_t* cfg, const voi
                                     mlra_stream_t stream);
 
 /*
+ * Workspace bytes mlra_decode_step needs for up to `batch` sequences on the
+ * current device: the mlra_decode_attn workspace (first, so that
+ * mlra_get_device_error reads the same error word) followed by the absorbed
+ * query, the latent output and staging room for the step's inputs and output.
+ */
+MLRA_API mlra_status_t mlra_step_workspace_size(const mlra_config_t* cfg, int32_t batch,
+                                                size_t* bytes);
+
+/*
+ * Steps 1, 2a, 2b and 3 in one call: absorb the query, split-KV attention,
+ * merge and output up-projection (Main Findings, the three absorbable steps),
+ * enqueued on `stream` in that order.  The result equals that of
+ * mlra_absorb_q -> mlra_decode_attn -> mlra_combine_out_proj bit for bit.
+ *   q_nope, q_rope, seqlens : as mlra_absorb_q / mlra_decode_attn
+ *   w_uk, w_uv              : as mlra_absorb_q / mlra_out_proj (device)
+ *   kv_cache, num_pages, page_table, max_pages : as mlra_decode_attn (device)
+ *   out      : [batch, n_heads, d_h] fp32 (written)
+ *   host_io  : 0 = q_nope, q_rope, seqlens and out are device memory;
+ *              1 = they are host memory: the call enqueues the transfer of
+ *              the inputs into the workspace, the kernels and the transfer of
+ *              out back to the host, and returns without waiting (out is
+ *              valid once `stream` has passed this call).  Page-locked host
+ *              memory mapped into the device's address space (cudaHostAlloc /
+ *              cudaMallocHost under unified addressing) is read by one
+ *              staging kernel and out is written by the projection kernel in
+ *              place; other host memory moves by cudaMemcpyAsync, which is
+ *              synchronous for pageable memory.  The host must not modify
+ *              the inputs or read out until the stream has passed the call.
+ *   workspace : >= mlra_step_workspace_size bytes, 256-byte aligned
+ * Errors as the three calls it makes; MLRA_ERR_INVALID_ARG for host_io not 0
+ * or 1.  batch = 0 launches nothing.
+ */
+MLRA_API mlra_status_t mlra_decode_step(const mlra_config_t* cfg, const void* q_nope,
+                                        const void* q_rope, const int32_t* seqlens, int32_t batch,
+                                        const void* w_uk, const void* w_uv, const void* kv_cache,
+                                        int64_t num_pages, const int32_t* page_table,
+                                        int32_t max_pages, float* out, int32_t host_io,
+                                        void* workspace, size_t workspace_bytes,
+                                        mlra_stream_t stream);
+
+/*
  * Cache write (the step before decode attention reads the cache; the paper
  * describes it in prose: Methodology, third paragraph, latent RMSNorm before
  * the up-projection; Main Findings, variance bullet, the KV latent scaled by
