@@ -30,7 +30,7 @@ BF16 = 1
 STATUS = {
     0: "MLRA_OK", 1: "MLRA_ERR_INVALID_ARG", 2: "MLRA_ERR_UNSUPPORTED", 3: "MLRA_ERR_ALIGNMENT",
     4: "MLRA_ERR_WORKSPACE", 5: "MLRA_ERR_CUDA", 6: "MLRA_ERR_BAD_PAGE", 7: "MLRA_ERR_TIMEOUT",
-    8: "MLRA_ERR_NO_DEVICE",
+    8: "MLRA_ERR_NO_DEVICE", 9: "MLRA_ERR_RANGE",
 }
 
 # Every symbol the C header declares (checked by the CPU tests).

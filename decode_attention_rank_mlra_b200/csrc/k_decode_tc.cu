@@ -27,6 +27,8 @@
 #include "tc_common.cuh"
 
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 namespace mlra {
 namespace {
@@ -549,11 +551,35 @@ cudaError_t launch_t(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t s
                     a);
 }
 
+// Head counts that are multiples of 128 go to the 128-head kernel
+// (k_decode_wide.cu); MLRA_TC_LAYOUT=rows keeps them on the kernel above
+// wherever it applies, for comparison.
+bool use_rows_layout() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MLRA_TC_LAYOUT");
+    v = (e && strcmp(e, "rows") == 0) ? 1 : 0;
+  }
+  return v == 1;
+}
+
+bool rows_supported(const mlra_config_t& c) {
+  if (c.d_cb != 128) return false;
+  if (c.n_heads != 16 && c.n_heads != 32 && c.n_heads != 64 && c.n_heads != 128) return false;
+  if (c.n_blocks != 1 && c.n_blocks != 2 && c.n_blocks != 4) return false;
+  return c.n_blocks % g_of(c) == 0;
+}
+
+bool use_wide(const mlra_config_t& c) {
+  return tc::wide_supported(c) && !(use_rows_layout() && rows_supported(c));
+}
+
 }  // namespace
 
 bool tc_supported(const mlra_config_t& c) {
   if (c.dtype != MLRA_BF16 || c.d_r != 64) return false;
   if (c.d_cb == 512) return tc::mla_supported(c);
+  if (use_wide(c)) return true;
   if (c.d_cb != 128) return false;
   if (c.n_heads != 16 && c.n_heads != 32 && c.n_heads != 64 && c.n_heads != 128) return false;
   if (c.n_blocks != 1 && c.n_blocks != 2 && c.n_blocks != 4) return false;
@@ -561,7 +587,9 @@ bool tc_supported(const mlra_config_t& c) {
 }
 
 void tc_grid(const mlra_config_t& c, int num_sms, int* n_groups, int* ctas_per_group) {
-  *n_groups = c.d_cb == 512 ? tc::mla_groups(c) : (c.n_blocks / g_of(c)) * (c.n_heads / hpc_of(c));
+  *n_groups = c.d_cb == 512 ? tc::mla_groups(c)
+              : use_wide(c) ? tc::wide_groups(c)
+                            : (c.n_blocks / g_of(c)) * (c.n_heads / hpc_of(c));
   *ctas_per_group = num_sms / *n_groups > 0 ? num_sms / *n_groups : 1;
 }
 
@@ -571,6 +599,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   cudaError_t e = tc::make_cache_map(a, &map);
   if (e != cudaSuccess) return e;
   if (c.d_cb == 512) return tc::launch_decode_tc_mla(map, a, st);
+  if (use_wide(c)) return tc::launch_decode_wide(map, a, st);
   switch (hpc_of(c) * 10 + g_of(c)) {
     case 164: return launch_t<4, 16>(map, a, st);
     case 162: return launch_t<2, 16>(map, a, st);

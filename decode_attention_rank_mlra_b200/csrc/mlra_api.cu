@@ -157,6 +157,7 @@ const char* mlra_status_string(mlra_status_t s) {
     case MLRA_ERR_BAD_PAGE: return "page id out of range (device)";
     case MLRA_ERR_TIMEOUT: return "bounded wait expired (device)";
     case MLRA_ERR_NO_DEVICE: return "no usable CUDA device";
+    case MLRA_ERR_RANGE: return "cache value outside the fp16 range of the tensor-core path (device)";
   }
   return "unknown status";
 }

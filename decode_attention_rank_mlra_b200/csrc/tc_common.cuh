@@ -84,5 +84,11 @@ inline bool mla_supported(const mlra_config_t& c) {
 inline int mla_groups(const mlra_config_t& c) { return (c.n_heads / 64) * 4; }
 cudaError_t launch_decode_tc_mla(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st);
 
+// Latent blocks of 128 channels, 128 heads x one branch per CTA
+// (k_decode_wide.cu): head counts that are multiples of 128.
+bool wide_supported(const mlra_config_t& c);
+int wide_groups(const mlra_config_t& c);
+cudaError_t launch_decode_wide(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st);
+
 }  // namespace tc
 }  // namespace mlra

@@ -68,7 +68,9 @@ typedef enum {
   MLRA_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed            */
   MLRA_ERR_BAD_PAGE = 6,     /* device: page id outside [0, num_pages)         */
   MLRA_ERR_TIMEOUT = 7,      /* device: a bounded wait expired                 */
-  MLRA_ERR_NO_DEVICE = 8     /* no usable sm_100 device                        */
+  MLRA_ERR_NO_DEVICE = 8,    /* no usable sm_100 device                        */
+  MLRA_ERR_RANGE = 9         /* device: a cache value of magnitude >= 65520 met
+                                the tensor-core kernel's fp16 output product   */
 } mlra_status_t;
 
 typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype_t;
