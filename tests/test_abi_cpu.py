@@ -45,6 +45,14 @@ def test_status_strings(L):
     assert mlra.status_string(0) == "ok"
     assert "page" in mlra.status_string(6)
     assert mlra.status_string(99) == "unknown status"
+    # every status the header declares has its own string and Python name
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "mlra.h")).read()
+    codes = {int(v): k for k, v in re.findall(r"(MLRA_\w+)\s*=\s*(\d+)", hdr.split("mlra_status_t;")[0])
+             if k.startswith("MLRA_ERR") or k == "MLRA_OK"}
+    assert codes[9] == "MLRA_ERR_RANGE"
+    for v, k in codes.items():
+        assert mlra.STATUS[v] == k
+        assert mlra.status_string(v) != "unknown status"
     assert L.mlra_version() == 10000
 
 

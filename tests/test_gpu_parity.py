@@ -144,6 +144,37 @@ def test_paged_tail_rows_never_matter():
         assert torch.equal(got[k], ref[k]), k
 
 
+def test_h128_paged_tail_rows_never_matter():
+    """The 128-head kernel converts each tile to fp16 in shared memory: rows past
+    seqlen hold NaN / inf and must still not change the result."""
+    inp = _small("mlra4_bf16_b8_h128_l131072_paged", 2, [70, 5])
+    ref = run_gpu(inp)
+    flat = inp.kv_cache.view(-1, inp.spec.D)
+    pt = inp.page_table.cpu()
+    flat[int(pt[0, 1]) * 64 + 6: int(pt[0, 1]) * 64 + 64] = float("nan")
+    flat[int(pt[1, 0]) * 64 + 5: int(pt[1, 0]) * 64 + 64] = float("inf")
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    for k in ("out", "o_lat", "lse"):
+        assert torch.equal(got[k], ref[k]), k
+
+
+def test_h128_cache_values_beyond_fp16_range_are_reported():
+    """The 128-head kernel carries the latent tile into P . C as fp16: a valid
+    cache value of magnitude >= 65520 is reported (MLRA_ERR_RANGE); 59904 is
+    still exact and matches the oracle."""
+    inp = _small("mlra4_bf16_b8_h128_l131072_paged", 2, [200, 90])
+    flat = inp.kv_cache.view(-1, inp.spec.D)
+    row = int(inp.page_table[0, 1].item()) * 64 + 3
+    flat[row, 5] = 60000.0          # bf16 59904: inside the fp16 range
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    compare_batch(inp, got, heads=[0, 1, 64, 127])
+    flat[row, 5] = 70000.0          # bf16 70144: outside
+    got = run_gpu(inp)
+    assert got["device_error"] == 9  # MLRA_ERR_RANGE
+
+
 def test_scores_rising_far_above_the_first_tile():
     """Later tiles score hundreds of log2 units above the first tile's max: the
     running reference point of the exponentials must move (no overflow)."""
