@@ -352,12 +352,12 @@ __global__ void __launch_bounds__(kThreadsW, 1)
           for (int k = 0; k < 32; ++k) z[k] = __uint_as_float(sv[k]);
         }
         const int valid = min(kTile, p.L - t * kTile);
-        // the scores are done with the tile: convert its latent boxes to fp16
-        // (row r: box r / 64, token row r % 64; this thread takes pieces
+        // The scores are done with the tile: its latent boxes are converted to
+        // fp16 (row r: box r / 64, token row r % 64; this thread takes pieces
         // 4x..4x+3 in swizzled order, so a quarter-warp touches different bank
         // groups).  Rows past the valid tokens are written as zeros here too,
         // so they never depend on which copy of the row this thread reads.
-        {
+        auto convert = [&]() {
           uint4* row = reinterpret_cast<uint4*>(stages + st * STAGE + (r >> 6) * kBoxBytes +
                                                 (r & 63) * 128);
           uint4 w[4];
@@ -384,7 +384,12 @@ __global__ void __launch_bounds__(kThreadsW, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) row[(4 * x + j) ^ (r & 7)] = w[j];
           if ((over & 0x80008000u) != 0) set_error(err, MLRA_ERR_RANGE);
-        }
+        };
+        // The two warps of a quadrant take the conversion and the exponentials
+        // in opposite orders, so one uses the conversion path while the other
+        // uses the XU pipe (the conversion has no barrier: both still meet the
+        // pair's barriers in the same order).
+        if (x == 0) convert();
         if (valid < kTile) {
 #pragma unroll
           for (int k = 0; k < 32; ++k)
@@ -425,6 +430,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
           }
         };
         exps();
+        if (x == 1) convert();
         // (ls bounds every P of this half: a P above 2^15 or a NaN fails the test)
         if (bar_red_or(pid, 64, !(ls <= kPMaxW) || !good)) {
           if (pair_fail(good)) { ok = false; break; }
