@@ -81,10 +81,11 @@ def test_batches_spanning_several_sequence_tiles(batch, fused):
 
 
 @pytest.mark.parametrize("fused", [False, True])
-@pytest.mark.parametrize("heads", [16, 32, 64])
+@pytest.mark.parametrize("heads", [16, 32, 64, 128])
 def test_mlra2_two_branches(heads, fused):
     """MLRA-2 (two latent blocks of 128, branch rescale 1/sqrt(2)): the same
-    kernels with two branches per CTA (h <= 32) or one (h = 64)."""
+    kernels with two branches per CTA (h <= 32), one (h = 64), or 128 heads of
+    one branch (h = 128)."""
     base = W.WORKLOADS["mlra4_bf16_b64_h32_l16384_paged"]
     seqlens = [1, 64, 700, 1300, 333]
     spec = W.scaled_down(base, len(seqlens), seqlen=max(seqlens), n_heads=heads, seed=23)
@@ -95,6 +96,21 @@ def test_mlra2_two_branches(heads, fused):
     assert got["device_error"] == 0
     assert mlra.decode_kernel_kind(config_of(spec)) == "tcgen05"
     compare_batch(inp, got, heads=sorted({0, heads // 2, heads - 1}))
+
+
+@pytest.mark.parametrize("heads", [128, 256])
+def test_single_128_channel_block_h128(heads):
+    """One latent block of 128 channels (n_blocks = 1, D = 192) with 128 and 256
+    heads: the 128-head kernel with one branch, one or two head groups."""
+    base = W.WORKLOADS["mlra4_bf16_b8_h128_l131072_paged"]
+    seqlens = [65, 1000, 129]
+    spec = W.scaled_down(base, len(seqlens), seqlen=max(seqlens), n_heads=heads, seed=29)
+    spec = spec.replace(n_blocks=1, name=spec.name + "_nb1")
+    assert spec.D == 192 and spec.branch_scale == 1.0
+    inp = W.make_inputs(spec, "cuda", seqlens=np.asarray(seqlens, np.int32))
+    got = run_gpu(inp, fused=True)
+    assert got["device_error"] == 0
+    compare_batch(inp, got, heads=sorted({0, 77, heads - 1}))
 
 
 def test_fused_projection_without_latent_outputs():
