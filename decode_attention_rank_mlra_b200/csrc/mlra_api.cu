@@ -142,6 +142,198 @@ StepLayout step_layout(const mlra_config_t& c, int batch, const Grid& g) {
   return s;
 }
 
+
+// ---------------------------------------------------------------------------
+// mlra_decode_step: one call's arguments, the transfers its host buffers need,
+// and the launches, replayed as a CUDA graph from the second call with the
+// same arguments on.
+struct StepCall {
+  mlra_config_t cfg;
+  const void *q_nope, *q_rope;
+  const int32_t* seqlens;
+  int32_t batch;
+  const void *w_uk, *w_uv, *kv_cache;
+  int64_t num_pages;
+  const int32_t* page_table;
+  int32_t max_pages;
+  float* out;
+  int32_t host_io;
+  void* workspace;
+  size_t workspace_bytes;
+  StepLayout S;
+  // resolved by resolve_step
+  const void *k_q_nope, *k_q_rope;  // what the kernels read
+  const int32_t* k_seqlens;
+  StageCopy staged[3];
+  int n_staged;
+  StageCopy copies_in[3];  // pageable inputs: copy-engine transfers
+  int n_copies_in;
+  float* dev_out;
+  bool copy_out;
+};
+
+// Host buffers: ranges the device can read in place (page-locked, mapped) move
+// in one staging launch, others by copy-engine transfers; the output is
+// written by the projection kernel straight into mapped host memory, else into
+// the workspace and copied back.
+void resolve_step(StepCall* c) {
+  char* ws = static_cast<char*>(c->workspace);
+  const size_t esz = c->cfg.dtype == MLRA_BF16 ? 2 : 4;
+  const size_t bh = size_t(c->batch) * c->cfg.n_heads;
+  c->k_q_nope = c->q_nope;
+  c->k_q_rope = c->q_rope;
+  c->k_seqlens = c->seqlens;
+  c->n_staged = c->n_copies_in = 0;
+  c->dev_out = c->out;
+  c->copy_out = false;
+  if (!c->host_io) return;
+  const void* src[3] = {c->q_nope, c->q_rope, c->seqlens};
+  const size_t off[3] = {c->S.q_nope, c->S.q_rope, c->S.seqlens};
+  const size_t len[3] = {bh * c->cfg.d_h * esz, bh * c->cfg.d_r * esz, size_t(c->batch) * 4};
+  for (int k = 0; k < 3; ++k) {
+    if (const void* d = mapped_host_range(src[k], len[k]))
+      c->staged[c->n_staged++] = StageCopy{d, ws + off[k], len[k]};
+    else
+      c->copies_in[c->n_copies_in++] = StageCopy{src[k], ws + off[k], len[k]};
+  }
+  c->k_q_nope = ws + c->S.q_nope;
+  c->k_q_rope = ws + c->S.q_rope;
+  c->k_seqlens = reinterpret_cast<const int32_t*>(ws + c->S.seqlens);
+  if (void* d = const_cast<void*>(mapped_host_range(c->out, bh * c->cfg.d_h * 4))) {
+    c->dev_out = static_cast<float*>(d);
+  } else {
+    c->dev_out = reinterpret_cast<float*>(ws + c->S.out);
+    c->copy_out = true;
+  }
+}
+
+mlra_status_t enqueue_step(const StepCall& c, cudaStream_t s) {
+  char* ws = static_cast<char*>(c.workspace);
+  mlra_stream_t stream = (mlra_stream_t)s;
+  for (int k = 0; k < c.n_copies_in; ++k)
+    if (cudaMemcpyAsync(c.copies_in[k].dst, c.copies_in[k].src, c.copies_in[k].bytes,
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return MLRA_ERR_CUDA;
+  if (c.n_staged > 0 && launch_stage(c.staged, c.n_staged, s) != cudaSuccess) return MLRA_ERR_CUDA;
+  float* q_abs = reinterpret_cast<float*>(ws + c.S.q_abs);
+  mlra_status_t st = mlra_absorb_q(&c.cfg, c.k_q_nope, c.w_uk, q_abs, c.batch, stream);
+  if (st != MLRA_OK) return st;
+  st = mlra_decode_attn(&c.cfg, q_abs, c.k_q_rope, c.kv_cache, c.num_pages, c.page_table,
+                        c.max_pages, c.k_seqlens, c.batch, c.workspace, c.S.attn, stream);
+  if (st != MLRA_OK) return st;
+  // The fused kernel needs no latent output; where it does not apply, the
+  // two-kernel fallback writes it to the workspace.
+  st = mlra_combine_out_proj(&c.cfg, c.workspace, c.S.attn, c.batch, c.w_uv, c.dev_out, nullptr,
+                             nullptr, stream);
+  if (st == MLRA_ERR_UNSUPPORTED)
+    st = mlra_combine_out_proj(&c.cfg, c.workspace, c.S.attn, c.batch, c.w_uv, c.dev_out,
+                               reinterpret_cast<float*>(ws + c.S.o_lat), nullptr, stream);
+  if (st != MLRA_OK || !c.copy_out) return st;
+  const size_t bytes = size_t(c.batch) * c.cfg.n_heads * c.cfg.d_h * 4;
+  return from_cuda(cudaMemcpyAsync(c.out, c.dev_out, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+// The graph cache: a call whose transfers are all kernels (device buffers, or
+// mapped host buffers) is keyed by everything it passes to the kernels.  The
+// first call with a key runs its launches directly (which also sets the
+// kernels' attributes), the second records them on a private stream and
+// instantiates the graph, later ones replay it: one launch instead of five.
+// The graph reads the lengths, queries and cache at replay time, so their
+// contents may change between calls; their addresses may not.  A stream that
+// the caller is capturing is never recorded into.  The cache holds a fixed
+// number of graphs and never evicts one (a replay may still be running).
+struct StepKey {
+  mlra_config_t cfg;
+  const void* p[10];
+  int64_t num_pages;
+  int32_t batch, max_pages, host_io, dev;
+  size_t workspace_bytes;
+};
+
+bool same_key(const StepKey& a, const StepKey& b) {
+  if (memcmp(&a.cfg, &b.cfg, sizeof(a.cfg)) != 0) return false;
+  for (int i = 0; i < 10; ++i)
+    if (a.p[i] != b.p[i]) return false;
+  return a.num_pages == b.num_pages && a.batch == b.batch && a.max_pages == b.max_pages &&
+         a.host_io == b.host_io && a.dev == b.dev && a.workspace_bytes == b.workspace_bytes;
+}
+
+struct StepGraph {
+  StepKey key;
+  int state;  // 1: seen once, 2: graph ready, -1: recording failed (run directly)
+  cudaGraphExec_t exec;
+};
+constexpr int kStepGraphs = 64;
+std::mutex g_step_mu;
+StepGraph g_step_graphs[kStepGraphs];
+int g_step_n = 0;
+cudaStream_t g_capture_stream[kMaxDevices] = {};
+
+mlra_status_t run_step(const StepCall& c, cudaStream_t s) {
+  const bool graphable = c.n_copies_in == 0 && !c.copy_out;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (!graphable || cudaStreamIsCapturing(s, &cs) != cudaSuccess ||
+      cs != cudaStreamCaptureStatusNone) {
+    (void)cudaGetLastError();
+    return enqueue_step(c, s);
+  }
+  StepKey k;
+  memset(&k, 0, sizeof(k));
+  k.cfg = c.cfg;
+  const void* ps[10] = {c.q_nope, c.q_rope, c.seqlens, c.w_uk, c.w_uv, c.kv_cache,
+                        c.page_table, c.out, c.workspace, c.dev_out};
+  for (int i = 0; i < 10; ++i) k.p[i] = ps[i];
+  k.num_pages = c.num_pages;
+  k.batch = c.batch;
+  k.max_pages = c.max_pages;
+  k.host_io = c.host_io;
+  k.workspace_bytes = c.workspace_bytes;
+  if (cudaGetDevice(&k.dev) != cudaSuccess || k.dev < 0 || k.dev >= kMaxDevices)
+    return enqueue_step(c, s);
+  StepGraph* e = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_step_mu);
+    for (int i = 0; i < g_step_n; ++i)
+      if (same_key(g_step_graphs[i].key, k)) e = &g_step_graphs[i];
+    if (e && e->state == 2) {
+      const cudaGraphExec_t exec = e->exec;
+      return from_cuda(cudaGraphLaunch(exec, s));
+    }
+    if (!e) {
+      if (g_step_n < kStepGraphs) {
+        g_step_graphs[g_step_n] = StepGraph{k, 1, nullptr};
+        ++g_step_n;
+      }
+      return enqueue_step(c, s);
+    }
+    if (e->state != 1) return enqueue_step(c, s);
+    // second call with this key: record it (under the lock, so that one thread
+    // records and the others wait for the graph)
+    cudaStream_t& cap = g_capture_stream[k.dev];
+    bool ok = cap != nullptr ||
+              cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking) == cudaSuccess;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    if (ok) ok = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    if (ok) {
+      const mlra_status_t rec = enqueue_step(c, cap);
+      const bool ended = cudaStreamEndCapture(cap, &graph) == cudaSuccess;
+      ok = rec == MLRA_OK && ended && graph != nullptr &&
+           cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+    }
+    if (graph) cudaGraphDestroy(graph);
+    (void)cudaGetLastError();
+    if (!ok) {
+      if (exec) cudaGraphExecDestroy(exec);
+      e->state = -1;
+      return enqueue_step(c, s);
+    }
+    e->exec = exec;
+    e->state = 2;
+    return from_cuda(cudaGraphLaunch(exec, s));
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -337,58 +529,26 @@ mlra_status_t mlra_decode_step(const mlra_config_t* cfg, const void* q_nope, con
   Grid g;
   st = plan_grid(*cfg, &g);
   if (st != MLRA_OK) return st;
-  const StepLayout S = step_layout(*cfg, batch, g);
-  if (workspace_bytes < S.total) return MLRA_ERR_WORKSPACE;
-  char* ws = static_cast<char*>(workspace);
-  cudaStream_t s = (cudaStream_t)stream;
-  const size_t esz = cfg->dtype == MLRA_BF16 ? 2 : 4;
-  const size_t bh = size_t(batch) * cfg->n_heads;
-  float* dev_out = out;
-  bool copy_out = false;
-  if (host_io) {
-    // Inputs: ranges the device can read in place move in one staging launch,
-    // any others (pageable memory) by copy-engine transfers.
-    const void* src[3] = {q_nope, q_rope, seqlens};
-    const size_t off[3] = {S.q_nope, S.q_rope, S.seqlens};
-    const size_t len[3] = {bh * cfg->d_h * esz, bh * cfg->d_r * esz, size_t(batch) * 4};
-    StageCopy staged[3];
-    int n_staged = 0;
-    for (int k = 0; k < 3; ++k) {
-      if (const void* d = mapped_host_range(src[k], len[k])) {
-        staged[n_staged++] = StageCopy{d, ws + off[k], len[k]};
-      } else if (cudaMemcpyAsync(ws + off[k], src[k], len[k], cudaMemcpyHostToDevice, s) !=
-                 cudaSuccess) {
-        return MLRA_ERR_CUDA;
-      }
-    }
-    if (n_staged > 0 && launch_stage(staged, n_staged, s) != cudaSuccess) return MLRA_ERR_CUDA;
-    q_nope = ws + S.q_nope;
-    q_rope = ws + S.q_rope;
-    seqlens = reinterpret_cast<const int32_t*>(ws + S.seqlens);
-    // Output: written by the projection kernel straight into mapped host
-    // memory, else into the workspace and copied back.
-    if (void* d = const_cast<void*>(mapped_host_range(out, bh * cfg->d_h * 4))) {
-      dev_out = static_cast<float*>(d);
-    } else {
-      dev_out = reinterpret_cast<float*>(ws + S.out);
-      copy_out = true;
-    }
-  }
-  float* q_abs = reinterpret_cast<float*>(ws + S.q_abs);
-  st = mlra_absorb_q(cfg, q_nope, w_uk, q_abs, batch, stream);
-  if (st != MLRA_OK) return st;
-  st = mlra_decode_attn(cfg, q_abs, q_rope, kv_cache, num_pages, page_table, max_pages, seqlens,
-                        batch, workspace, S.attn, stream);
-  if (st != MLRA_OK) return st;
-  // The fused kernel needs no latent output; where it does not apply, the
-  // two-kernel fallback writes it to the workspace.
-  st = mlra_combine_out_proj(cfg, workspace, S.attn, batch, w_uv, dev_out, nullptr, nullptr,
-                             stream);
-  if (st == MLRA_ERR_UNSUPPORTED)
-    st = mlra_combine_out_proj(cfg, workspace, S.attn, batch, w_uv, dev_out,
-                               reinterpret_cast<float*>(ws + S.o_lat), nullptr, stream);
-  if (st != MLRA_OK || !copy_out) return st;
-  return from_cuda(cudaMemcpyAsync(out, dev_out, bh * cfg->d_h * 4, cudaMemcpyDeviceToHost, s));
+  StepCall c;
+  c.cfg = *cfg;
+  c.q_nope = q_nope;
+  c.q_rope = q_rope;
+  c.seqlens = seqlens;
+  c.batch = batch;
+  c.w_uk = w_uk;
+  c.w_uv = w_uv;
+  c.kv_cache = kv_cache;
+  c.num_pages = num_pages;
+  c.page_table = page_table;
+  c.max_pages = max_pages;
+  c.out = out;
+  c.host_io = host_io;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  c.S = step_layout(*cfg, batch, g);
+  if (workspace_bytes < c.S.total) return MLRA_ERR_WORKSPACE;
+  resolve_step(&c);
+  return run_step(c, (cudaStream_t)stream);
 }
 
 mlra_status_t mlra_cache_append(const mlra_config_t* cfg, const void* c_new,

@@ -133,3 +133,59 @@ def test_step_workspace_holds_decode_workspace():
     for b in (1, 64, 300):
         assert mlra.step_workspace_size(cfg, b) >= mlra.workspace_size(cfg, b) \
             + 2 * b * cfg.n_heads * cfg.n_blocks * cfg.d_cb * 4
+
+
+@pytest.mark.parametrize("host", [False, True])
+def test_repeated_steps_with_new_lengths(host):
+    """The same buffers called again and again (the first call runs directly,
+    the second is recorded, later ones replay the recording) with new sequence
+    lengths each time: every result equals the separate calls on those lengths."""
+    inp = _inputs("mlra4_bf16_b64_h32_l16384_paged", [1999] * 4)  # pages for 1999 tokens each
+    base = [700, 64, 1999, 3]
+    cfg = config_of(inp.spec)
+    dec = mlra.Decoder(cfg, inp.spec.batch, inp.device)
+    ref_dec = mlra.Decoder(cfg, inp.spec.batch, inp.device)
+    if host:
+        qn, qr = inp.q_nope.cpu().pin_memory(), inp.q_rope.cpu().pin_memory()
+        sl = inp.seqlens.cpu().pin_memory()
+        out = torch.empty(dec.out.shape, dtype=torch.float32).pin_memory()
+    else:
+        qn, qr, sl = inp.q_nope, inp.q_rope, inp.seqlens.clone()
+        out = dec.out
+    for i, lens in enumerate([base, [5, 1999, 64, 700], [1, 1, 1, 1], [640, 0, 129, 1000],
+                              base]):
+        sl.copy_(torch.tensor(lens, dtype=torch.int32))
+        d_sl = sl.to(inp.device)
+        dec.step(qn, qr, sl, inp.w_uk, inp.w_uv, inp.kv_cache, inp.page_table, _max_pages(inp),
+                 out=out)
+        ref_dec.run(inp.q_nope, inp.q_rope, inp.w_uk, inp.w_uv, inp.kv_cache, inp.page_table,
+                    d_sl, _max_pages(inp), fused=True)
+        torch.cuda.synchronize()
+        assert mlra.get_device_error(dec.workspace) == 0
+        assert torch.equal(out.cpu(), ref_dec.out.cpu()), f"call {i}"
+
+
+def test_step_inside_a_caller_graph():
+    """A caller that captures the step into its own CUDA graph gets the launches
+    themselves in that graph (the library does not record into a capturing
+    stream); replays match the direct result."""
+    inp = _inputs("mlra4_bf16_b16_h16_l4096_contig", [900, 64, 1, 333])
+    cfg = config_of(inp.spec)
+    dec = mlra.Decoder(cfg, inp.spec.batch, inp.device)
+    args = (inp.q_nope, inp.q_rope, inp.seqlens, inp.w_uk, inp.w_uv, inp.kv_cache,
+            inp.page_table, _max_pages(inp))
+    ref = dec.step(*args).clone()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            dec.step(*args)
+    torch.cuda.current_stream().wait_stream(s)
+    dec.out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(dec.out, ref)
+    assert mlra.get_device_error(dec.workspace) == 0
