@@ -223,6 +223,13 @@ MLRA_API mlra_status_t mlra_step_workspace_size(const mlra_config_t* cfg, int32_
  *   workspace : >= mlra_step_workspace_size bytes, 256-byte aligned
  * Errors as the three calls it makes; MLRA_ERR_INVALID_ARG for host_io not 0
  * or 1.  batch = 0 launches nothing.
+ * Repeated calls: a call whose transfers are all kernels (device buffers, or
+ * mapped host buffers) is recorded as a CUDA graph the second time the same
+ * pointers, sizes and configuration are passed, and later calls replay it (one
+ * graph launch instead of five kernel launches; the contents of every buffer
+ * may change between calls, as with direct launches).  Nothing is recorded
+ * while `stream` is being captured by the caller.  The library keeps up to 64
+ * such graphs per process for its lifetime.
  */
 MLRA_API mlra_status_t mlra_decode_step(const mlra_config_t* cfg, const void* q_nope,
                                         const void* q_rope, const int32_t* seqlens, int32_t batch,
