@@ -80,6 +80,18 @@ bool use_proj_tc(const mlra_config_t& c) {
   return device_is_sm100(dev);
 }
 
+// MLRA_TEST_STALL_TILE=<k>: tests of the failure path only (see
+// DecodeArgs::stall_tile).  Read once per process.
+int test_stall_tile() {
+  static int v = -2;
+  if (v == -2) {
+    const char* e = getenv("MLRA_TEST_STALL_TILE");
+    v = e ? atoi(e) : -1;
+    if (v < 0) v = -1;
+  }
+  return v;
+}
+
 struct Grid { int kind, n_groups, ctas_per_group; };
 
 mlra_status_t plan_grid(const mlra_config_t& c, Grid* g) {
@@ -436,6 +448,7 @@ mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, con
   a.L = L;
   a.ctas_per_group = g.ctas_per_group;
   a.n_groups = g.n_groups;
+  a.stall_tile = test_stall_tile();
   e = (g.kind == 1) ? launch_decode_tc(a, s) : launch_decode_simt(a, s);
   return from_cuda(e);
 }

@@ -267,6 +267,11 @@ struct DecodeArgs {
   WsLayout L;
   int32_t ctas_per_group;
   int32_t n_groups;
+  // Test of the failure path: the TMA producer of CTA 0 leaves the full
+  // barrier of this tile (its count in that CTA's stream) unsignalled, so the
+  // MMA warp's bounded wait runs out (MLRA_ERR_TIMEOUT).  -1: none.  Set only
+  // from MLRA_TEST_STALL_TILE; honoured by the head-rows kernel.
+  int32_t stall_tile = -1;
 };
 
 }  // namespace mlra

@@ -1,0 +1,53 @@
+"""GPU failure path: a wait that runs out ends with an error status, not a hang.
+
+The attention kernel bounds every mbarrier wait (2 s).  MLRA_TEST_STALL_TILE=k
+makes the TMA producer of CTA 0 leave the full barrier of its k-th tile
+unsignalled, so the MMA warp's wait runs out: the call must report
+MLRA_ERR_TIMEOUT in the workspace's error word within seconds, and the CUDA
+context must stay usable.  Runs in a child process (the variable is read once
+per process).
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r"""
+import sys, time, numpy as np, torch
+sys.path.insert(0, ROOT); sys.path.insert(0, ROOT + "/tests")
+import decode_attention_rank_mlra_b200 as mlra
+import workloads as W
+from parity_util import config_of
+spec = W.scaled_down(W.WORKLOADS["mlra4_bf16_b16_h16_l4096_contig"], 2, seqlen=300, seed=3)
+inp = W.make_inputs(spec, "cuda", seqlens=np.asarray([300, 200], np.int32))
+cfg = config_of(spec)
+dec = mlra.Decoder(cfg, 2, inp.device)
+mlra.absorb_q(cfg, inp.q_nope, inp.w_uk, dec.q_abs)
+t0 = time.time()
+mlra.decode_attn(cfg, dec.q_abs, inp.q_rope, inp.kv_cache, None, inp.seqlens, inp.max_len,
+                 dec.workspace)
+err = mlra.get_device_error(dec.workspace)
+dt = time.time() - t0
+# the context is still usable: a library kernel and a torch kernel run and agree
+q2 = mlra.absorb_q(cfg, inp.q_nope, inp.w_uk)
+ok = bool(torch.equal(q2, dec.q_abs)) and float((inp.q_nope.float() * 0 + 1).sum()) > 0
+torch.cuda.synchronize()
+print(f"status {err} seconds {dt:.2f} usable {ok}")
+""".replace("ROOT", repr(ROOT))
+
+
+def test_bounded_wait_reports_timeout():
+    env = dict(os.environ, MLRA_TEST_STALL_TILE="0")
+    r = subprocess.run([sys.executable, "-c", CHILD], env=env, cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = [l for l in r.stdout.splitlines() if l.startswith("status")][-1]
+    fields = line.split()
+    assert fields[1] == "7", line          # MLRA_ERR_TIMEOUT
+    assert float(fields[3]) < 60.0, line   # bounded: ~2 s of wait plus draining
+    assert fields[5] == "True", line
