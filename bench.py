@@ -350,6 +350,10 @@ def run_ours(args):
                                                   dec.workspace),
         "combine_out_proj": lambda i: mlra.combine_out_proj(cfg, dec.workspace, B, inp.w_uv,
                                                             dec.out, dec.o_latent, dec.lse),
+        # the same two steps unfused (the step above uses the fused call)
+        "splitkv_combine": lambda i: mlra.splitkv_combine(cfg, dec.workspace, B, dec.o_latent,
+                                                          dec.lse),
+        "out_proj": lambda i: mlra.out_proj(cfg, dec.o_latent, inp.w_uv, dec.out),
         # the cache-write step (not part of the step above): every sequence's
         # last row rewritten from a normalised latent and a rotated RoPE key
         "cache_append": lambda i: mlra.cache_append(cfg, app_c, app_kr, app_gamma, 2.0,
