@@ -7,17 +7,20 @@
 // n_blocks = 1: z_t = (q_abs . c[t] + q_rope . k_rope[t]) * scale,
 // o = softmax(z) . c, lse = log sum exp z, per head and split.
 //
-// How.  With 64 heads a CTA's MMA rows are (head, hi|lo) = 128, and the
-// queries (512 + 64 channels as bf16 hi/lo pairs) take 288 of the 512 TMEM
-// columns, so the 512-wide output cannot sit next to them: a CTA owns one
-// 128-feature quarter of the output.  The four quarter CTAs of a head group
-// compute the same scores (bit for bit: same operands, same MMA order) and
-// each multiplies the probabilities by its quarter of the tile.
+// How.  With 64 heads a CTA's MMA rows are (head, hi|lo) = 128.  The 512-wide
+// output does not fit TMEM beside the queries, so a CTA owns one 256-feature
+// half of the output, and the two half CTAs of a head group compute the same
+// scores (bit for bit: same operands, same MMA order).  TMEM holds the hi/lo
+// queries of latent channels 0-255 (128 columns), the RoPE query (32), S (64)
+// and the O half (256); the queries of channels 256-511 sit in shared memory
+// (64 KB, K-major, 128-byte swizzle) as the A operand of the second half of
+// the scores.
 //  * warp 4: TMA of the nine 64-column boxes of a 64-token tile (8 latent +
-//    RoPE) into a 3-stage ring;
-//  * warp 5: S = Q C^T over K = 512 + 64 (36 MMAs of M = 128, N = 64, A in
-//    TMEM), then, once the softmax has written P over S, O += P C_q over the
-//    quarter's two boxes (MN-major B, N = 128);
+//    RoPE) into a 2-stage ring;
+//  * warp 5: S = Q C^T over K = 512 + 64 (36 MMAs of M = 128, N = 64: 16 with
+//    A in TMEM, 16 with A in shared memory, 4 for RoPE), then, once the
+//    softmax has written P over S, O += P C_q over the half's four boxes
+//    (MN-major B, two MMA groups of N = 128);
 //  * warps 0-3: the softmax of the hi / lo rows exactly as in k_decode_tc.cu.
 // S has a single 64-column buffer (TMEM is full), so the QK of tile i+1 is
 // issued right after the PV of tile i.
@@ -36,14 +39,16 @@ constexpr int kHeads = 64;             // heads per CTA (128 MMA rows with hi / 
 constexpr int kLat = 512;              // latent channels
 constexpr int kBoxes = kLat / kBoxCols + 1;  // 8 latent boxes + RoPE
 constexpr int kStage = kBoxes * kBoxBytes;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQ = 0;          // q_abs hi / lo rows: 256 columns
-constexpr uint32_t kColQr = 256;       // q_rope rows: 32 columns
-constexpr uint32_t kColS = 288;        // S / P: 64 columns
-constexpr uint32_t kColO = 384;        // O quarter: 128 columns
+constexpr uint32_t kColQ = 0;          // q_abs hi / lo rows, channels 0-255: 128 columns
+constexpr uint32_t kColQr = 128;       // q_rope rows: 32 columns
+constexpr uint32_t kColS = 160;        // S / P: 64 columns
+constexpr uint32_t kColO = 224;        // O half: two 128-feature quarters, 256 columns
+constexpr int kQsChunk = 128 * 128;    // 128 rows x 64 channels of bf16
+constexpr int kQsBytes = 4 * kQsChunk; // q_abs hi / lo rows, channels 256-511
 constexpr int kBars = 2 * kStages + 6;
-constexpr int kSmem = 1024 + kStages * kStage + kBars * 8 + 64;
+constexpr int kSmem = 1024 + kQsBytes + kStages * kStage + kBars * 8 + 64;
 static_assert(kSmem <= kSmemLimit, "shared memory");
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -51,8 +56,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* stages = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStage);
+  uint8_t* q_sm = smem;                  // queries of channels 256-511
+  uint8_t* stages = smem + kQsBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * kStage);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_addr(bars);
@@ -99,8 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int H = a.cfg.n_heads;
   const int grp = blockIdx.x / a.ctas_per_group;
   const int c = blockIdx.x % a.ctas_per_group;
-  const int fq = grp & 3;                 // output quarter: features 128 fq ..
-  const int head0 = (grp >> 2) * kHeads;  // first head of the CTA's head group
+  const int fh = grp & 1;                 // output half: features 256 fh ..
+  const int head0 = (grp >> 1) * kHeads;  // first head of the CTA's head group
   __shared__ int plan_sm[12], scan_sm[kThreads / 32 + 1];
   plan_first_pieces<kThreads>(a.seqlens, a.batch, a.cap, a.ctas_per_group, c, plan_sm, scan_sm);
   const int total = plan_sm[0], share = plan_sm[1];
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase0 = smem_addr(stages);
     const uint64_t dK = smem_desc(sbase0, 16, 1024, kSwizzle128B);
     const uint64_t dMN = smem_desc(sbase0, kBoxBytes, 1024, kSwizzle128B);
+    const uint64_t dQs = smem_desc(smem_addr(q_sm), 16, 1024, kSwizzle128B);
     Piece p;
     int it = 0, piece = 0;
     bool ok = true;
@@ -181,12 +188,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         tc_fence_after();
         const uint64_t d = dK + uint64_t((st * kStage) >> 4);
-        // S = Q_lat C^T (32 K-steps over the 8 latent boxes) + Q_rope K_rope^T
+        // S = Q_lat C^T (32 K-steps over the 8 latent boxes: channels 0-255
+        // with A in TMEM, 256-511 with A in shared memory) + Q_rope K_rope^T
 #pragma unroll
-        for (int k = 0; k < kLat / 16; ++k)
+        for (int k = 0; k < 16; ++k)
           mma_ts_warp(tmem + kColS, tmem + kColQ + 8 * k,
                       d + uint64_t(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), kIdescQK,
                       k > 0 ? 1u : 0u, 0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int k = 16; k < kLat / 16; ++k)
+          mma_ss_warp(tmem + kColS,
+                      dQs + uint64_t((((k - 16) >> 2) * kQsChunk + ((k - 16) & 3) * 32) >> 4),
+                      d + uint64_t(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4), kIdescQK, 1u);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           mma_ts_warp(tmem + kColS, tmem + kColQr + 8 * k,
@@ -196,11 +209,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O_q += P C_q once the probabilities are over S
         if (!wait_bar(PREADY, it & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t dv = dMN + uint64_t((st * kStage + 2 * fq * kBoxBytes) >> 4);
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          mma_ts_warp(tmem + kColO, tmem + kColS + 8 * k, dv + uint64_t((k * 16 * 128) >> 4),
-                      kIdescPV, (t == p.t0 && k == 0) ? 0u : 1u, 0u, 0u, 0u, 0u);
+        for (int qq = 0; qq < 2; ++qq) {
+          const uint64_t dv =
+              dMN + uint64_t((st * kStage + 2 * (2 * fh + qq) * kBoxBytes) >> 4);
+#pragma unroll
+          for (int k = 0; k < kTile / 16; ++k)
+            mma_ts_warp(tmem + kColO + 128 * qq, tmem + kColS + 8 * k,
+                        dv + uint64_t((k * 16 * 128) >> 4), kIdescPV,
+                        (t == p.t0 && k == 0) ? 0u : 1u, 0u, 0u, 0u, 0u);
+        }
         mma_commit_warp(EMPTY(st));
         mma_commit_warp(PVDONE);
       }
@@ -233,48 +251,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto qr_row = [&](const Piece& pc) {
       return reinterpret_cast<const uint4*>(q_rope + (size_t(pc.s) * H + head) * 64);
     };
-    // Thread t converts channels [0, 256) of head t's query, thread t + 16
-    // channels [256, 512); the split stores place both halves in the hi row and
-    // in the lo row.  Two rounds of 32 loads.
+    // Thread (warp, lane) fills MMA row 32 warp + lane: the hi (x = 0) or lo
+    // (x = 1) bf16 part of its head's query.  Channels 0-255 go to TMEM (32x32b
+    // stores: a thread writes its own lane), channels 256-511 to the shared-
+    // memory A operand: four 16 KB chunks of 64 channels, K-major with the
+    // 128-byte swizzle (16-byte unit u of row r at u ^ (r & 7)).  The previous
+    // piece's QK MMAs, the only readers of either, are complete when this runs.
+    uint8_t* const q_srow = q_sm + (4 * warp + (lane >> 3)) * 1024 + (lane & 7) * 128;
     auto write_q = [&](const Piece& pc) {
-      const float4* q = q_row(pc) + 64 * x;
+      const float4* q = q_row(pc);
 #pragma unroll 1
-      for (int r = 0; r < 2; ++r) {
-        float4 f[32];
+      for (int r = 0; r < 8; ++r) {  // 64 channels per round
+        float4 f[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) f[j] = __ldg(q + 32 * r + j);
+        for (int j = 0; j < 16; ++j) f[j] = __ldg(q + 16 * r + j);
+        uint32_t w[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t hi[32], lo[32];
+        for (int j = 0; j < 16; ++j) {
+          const float v[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
+          float u[4];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float4 v4 = f[16 * h + j];
-            const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-            float w[4];
+          for (int e = 0; e < 4; ++e)
+            u[e] = x ? v[e] - __bfloat162float(__float2bfloat16_rn(v[e])) : v[e];
+          w[2 * j] = pack_bf16(u[0], u[1]);
+          w[2 * j + 1] = pack_bf16(u[2], u[3]);
+        }
+        if (r < 4) {
+          tmem_st32(row_t + kColQ + 32 * r, w);
+        } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) w[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
-            hi[2 * j] = pack_bf16(v[0], v[1]);
-            hi[2 * j + 1] = pack_bf16(v[2], v[3]);
-            lo[2 * j] = pack_bf16(w[0], w[1]);
-            lo[2 * j + 1] = pack_bf16(w[2], w[3]);
-          }
-          const uint32_t col = kColQ + 32 * (2 * r + h);
-          tmem_st_x2_32<128>(hi_t + col, hi);
-          tmem_st_x2_32<128>(lo_t + col, lo);
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(q_srow + (r - 4) * kQsChunk + ((k ^ (lane & 7)) << 4)) =
+                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
-      const uint4* qr = qr_row(pc) + 4 * x;
-      uint32_t rr[16];
+      // RoPE query: the hi row holds it, the lo row zeros
+      uint32_t rr[32];
+      if (x == 0) {
+        const uint4* qr = qr_row(pc);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 u = __ldg(qr + j);
-        rr[4 * j] = u.x; rr[4 * j + 1] = u.y; rr[4 * j + 2] = u.z; rr[4 * j + 3] = u.w;
+        for (int j = 0; j < 8; ++j) {
+          const uint4 u = __ldg(qr + j);
+          rr[4 * j] = u.x; rr[4 * j + 1] = u.y; rr[4 * j + 2] = u.z; rr[4 * j + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) rr[j] = 0u;
       }
-      tmem_st_x2_16<16>(hi_t + kColQr, rr);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) rr[j] = 0u;
-      tmem_st_x2_16<16>(lo_t + kColQr, rr);
+      tmem_st32(row_t + kColQr, rr);
       tmem_wait_st();
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(QREADY);
@@ -357,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_bar_warp(PVDONE, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 8; ++ch) {
               uint32_t r[32];
               tmem_ld32(row_t + kColO + 32 * ch, r);
               tmem_wait_ld();
@@ -381,17 +407,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t + 1 == p.t1 && has_next) write_q(pn);
       }
       if (!ok) break;
-      // ---- epilogue: o = (O_hi + O_lo) / l for the quarter, lse
+      // ---- epilogue: o = (O_hi + O_lo) / l for the half, lse
       if (!wait_bar_warp(PVDONE, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
       const float l_tot = l + __shfl_xor_sync(0xffffffffu, l, 16);
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      float* dst = o_part + (size_t(p.slot) * H + head) * kLat + 128 * fq;
+      float* dst = o_part + (size_t(p.slot) * H + head) * kLat + 256 * fh;
 #pragma unroll 1
-      for (int j = 0; j < 2; ++j) {
+      for (int j = 0; j < 4; ++j) {
         uint32_t oh[32], ol[32];
-        tmem_ld_x2_32<64>(hi_t + kColO + 32 * j, oh);
-        tmem_ld_x2_32<64>(lo_t + kColO + 32 * j, ol);
+        tmem_ld_x2_32<128>(hi_t + kColO + 32 * j, oh);
+        tmem_ld_x2_32<128>(lo_t + kColO + 32 * j, ol);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -399,11 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             o8[e] = (__uint_as_float(oh[8 * k + e]) + __uint_as_float(ol[8 * k + e])) * inv;
-          st_global_v8(dst + 64 * x + 32 * j + 8 * k, o8);
+          st_global_v8(dst + 128 * x + 32 * j + 8 * k, o8);
         }
       }
-      // the four quarter CTAs hold the same m and l: quarter 0 writes the lse
-      if (fq == 0 && x == 0)
+      // the two half CTAs hold the same m and l: half 0 writes the lse
+      if (fh == 0 && x == 0)
         lse_part[size_t(p.slot) * H + head] =
             l_tot > 0.f ? (m + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
       if (!has_next) break;

@@ -77,11 +77,11 @@ inline cudaError_t make_cache_map(const DecodeArgs& a, CUtensorMap* map) {
 }
 
 // MLA (one latent block of 512, k_decode_tc_mla.cu): CTAs of 64 heads x one
-// 128-feature quarter of the latent output.
+// 256-feature half of the latent output.
 inline bool mla_supported(const mlra_config_t& c) {
   return c.n_blocks == 1 && c.d_cb == 512 && c.d_r == 64 && c.n_heads % 64 == 0;
 }
-inline int mla_groups(const mlra_config_t& c) { return (c.n_heads / 64) * 4; }
+inline int mla_groups(const mlra_config_t& c) { return (c.n_heads / 64) * 2; }
 cudaError_t launch_decode_tc_mla(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st);
 
 // Latent blocks of 128 channels, 128 heads x one branch per CTA
