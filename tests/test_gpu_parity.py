@@ -191,6 +191,27 @@ def test_h128_cache_values_beyond_fp16_range_are_reported():
     assert got["device_error"] == 9  # MLRA_ERR_RANGE
 
 
+def test_mla_tile_boundaries():
+    """MLA: lengths on both sides of the 32- and 64-token boundaries (a last
+    tile holding 1, 31, 32, 33 or 63 tokens), then NaN / inf in the rows past
+    seqlen must leave every output unchanged."""
+    seqlens = [1, 31, 32, 33, 63, 64, 65, 96, 97, 128]
+    inp = _small("mla_bf16_b8_h128_l131072_paged", len(seqlens), seqlens, seed=31)
+    ref = run_gpu(inp)
+    assert ref["device_error"] == 0
+    compare_batch(inp, ref, heads=[0, 37, 64, 127])
+    flat = inp.kv_cache.view(-1, inp.spec.D)
+    pt = inp.page_table.cpu()
+    for s, L in enumerate(seqlens):
+        if L % 64:
+            r0 = int(pt[s, L // 64]) * 64
+            flat[r0 + L % 64: r0 + 64] = float("nan") if s % 2 else float("inf")
+    got = run_gpu(inp)
+    assert got["device_error"] == 0
+    for k in ("out", "o_lat", "lse"):
+        assert torch.equal(got[k], ref[k]), k
+
+
 def test_scores_rising_far_above_the_first_tile():
     """Later tiles score hundreds of log2 units above the first tile's max: the
     running reference point of the exponentials must move (no overflow)."""
