@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             row = p.s * a.max_pages + t * kTile;
           }
+          if (it == a.stall_tile && blockIdx.x == 0) continue;  // failure-path test only
           mbar_arrive_expect_tx(FULL(st), kStage);
           const uint32_t dst = smem_addr(stages + st * kStage);
 #pragma unroll

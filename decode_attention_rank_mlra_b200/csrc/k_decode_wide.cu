@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
           } else {
             row = p.s * a.max_pages + t * kTile;
           }
+          if (it == a.stall_tile && blockIdx.x == 0) continue;  // failure-path test only
           mbar_arrive_expect_tx(FULL(st), STAGE);
           const uint32_t dst = smem_addr(stages + st * STAGE);
           tma_load_2d_hint(dst, &tmap, branch * 128, row, FULL(st), evict_first);

@@ -1,11 +1,13 @@
 """GPU failure path: a wait that runs out ends with an error status, not a hang.
 
-The attention kernel bounds every mbarrier wait (2 s).  MLRA_TEST_STALL_TILE=k
+The attention kernels bound every mbarrier wait (2 s).  MLRA_TEST_STALL_TILE=k
 makes the TMA producer of CTA 0 leave the full barrier of its k-th tile
-unsignalled, so the MMA warp's wait runs out: the call must report
-MLRA_ERR_TIMEOUT in the workspace's error word within seconds, and the CUDA
-context must stay usable.  Runs in a child process (the variable is read once
-per process).
+unsignalled, so the MMA warp's wait runs out and the other roles leave on the
+abort flag: the call must report MLRA_ERR_TIMEOUT in the workspace's error word
+within seconds, and the CUDA context must stay usable.  One child process per
+attention kernel (the variable is read once per process): the head-rows kernel
+(16 heads), the 128-head kernel (whose paired softmax warps leave a failed wait
+together through votes at their named barrier) and the MLA kernel.
 """
 import os
 import subprocess
@@ -23,13 +25,14 @@ sys.path.insert(0, ROOT); sys.path.insert(0, ROOT + "/tests")
 import decode_attention_rank_mlra_b200 as mlra
 import workloads as W
 from parity_util import config_of
-spec = W.scaled_down(W.WORKLOADS["mlra4_bf16_b16_h16_l4096_contig"], 2, seqlen=300, seed=3)
+spec = W.scaled_down(W.WORKLOADS[NAME], 2, seqlen=300, seed=3)
 inp = W.make_inputs(spec, "cuda", seqlens=np.asarray([300, 200], np.int32))
+mp = inp.page_table.shape[1] if inp.page_table is not None else inp.max_len
 cfg = config_of(spec)
 dec = mlra.Decoder(cfg, 2, inp.device)
 mlra.absorb_q(cfg, inp.q_nope, inp.w_uk, dec.q_abs)
 t0 = time.time()
-mlra.decode_attn(cfg, dec.q_abs, inp.q_rope, inp.kv_cache, None, inp.seqlens, inp.max_len,
+mlra.decode_attn(cfg, dec.q_abs, inp.q_rope, inp.kv_cache, inp.page_table, inp.seqlens, mp,
                  dec.workspace)
 err = mlra.get_device_error(dec.workspace)
 dt = time.time() - t0
@@ -41,9 +44,13 @@ print(f"status {err} seconds {dt:.2f} usable {ok}")
 """.replace("ROOT", repr(ROOT))
 
 
-def test_bounded_wait_reports_timeout():
+@pytest.mark.parametrize("name", ["mlra4_bf16_b16_h16_l4096_contig",
+                                  "mlra4_bf16_b8_h128_l131072_paged",
+                                  "mla_bf16_b8_h128_l131072_paged"])
+def test_bounded_wait_reports_timeout(name):
     env = dict(os.environ, MLRA_TEST_STALL_TILE="0")
-    r = subprocess.run([sys.executable, "-c", CHILD], env=env, cwd=ROOT, capture_output=True,
+    child = CHILD.replace("NAME", repr(name))
+    r = subprocess.run([sys.executable, "-c", child], env=env, cwd=ROOT, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     line = [l for l in r.stdout.splitlines() if l.startswith("status")][-1]
