@@ -75,3 +75,33 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
     res = bench.run_reference(Args())
     assert res["impl"] == "reference" and res["value"] > 0
     assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_traffic_only_for_the_captured_kernel_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu capture only while the
+    attention kernels' sources hash to the captured ones; an edited source makes
+    it null with the reason, and an unknown workload has no figure."""
+    import json
+    import shutil
+
+    import bench
+    got, src = bench.measured_traffic("mlra4_bf16_b16_h16_l4096_contig")
+    assert isinstance(got, int) and got > 0, src
+    # a copy of the tree's profiles and kernel sources with one source edited
+    fake = tmp_path / "root"
+    (fake / "profiles").mkdir(parents=True)
+    shutil.copy(os.path.join(ROOT, "profiles", "traffic.json"), fake / "profiles")
+    csrc = fake / "decode_attention_rank_mlra_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    names = json.load(open(fake / "profiles" / "traffic.json"))["sources"]
+    for n in names:
+        shutil.copy(os.path.join(ROOT, "decode_attention_rank_mlra_b200", "csrc", n), csrc)
+    monkeypatch.setattr(bench, "ROOT", str(fake))
+    got, src = bench.measured_traffic("mlra4_bf16_b16_h16_l4096_contig")
+    assert isinstance(got, int), src
+    got, src = bench.measured_traffic("no_such_workload")
+    assert got is None and "no ncu capture" in src
+    with open(csrc / names[0], "a") as f:
+        f.write("\n// edited\n")
+    got, src = bench.measured_traffic("mlra4_bf16_b16_h16_l4096_contig")
+    assert got is None and "changed" in src
