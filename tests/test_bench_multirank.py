@@ -78,30 +78,31 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
 
 
 def test_traffic_only_for_the_captured_kernel_sources(tmp_path, monkeypatch):
-    """roofline.traffic comes from the committed ncu capture only while the
-    attention kernels' sources hash to the captured ones; an edited source makes
-    it null with the reason, and an unknown workload has no figure."""
+    """roofline.traffic comes from an ncu capture only while the attention
+    kernels' sources hash to the captured ones: a tree whose capture matches
+    gives the figure, an unknown workload none, an edited source none."""
+    import hashlib
     import json
     import shutil
 
     import bench
-    got, src = bench.measured_traffic("mlra4_bf16_b16_h16_l4096_contig")
-    assert isinstance(got, int) and got > 0, src
-    # a copy of the tree's profiles and kernel sources with one source edited
+    names = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["sources"]
     fake = tmp_path / "root"
     (fake / "profiles").mkdir(parents=True)
-    shutil.copy(os.path.join(ROOT, "profiles", "traffic.json"), fake / "profiles")
     csrc = fake / "decode_attention_rank_mlra_b200" / "csrc"
     csrc.mkdir(parents=True)
-    names = json.load(open(fake / "profiles" / "traffic.json"))["sources"]
+    h = hashlib.sha256()
     for n in names:
         shutil.copy(os.path.join(ROOT, "decode_attention_rank_mlra_b200", "csrc", n), csrc)
+        h.update((csrc / n).read_bytes())
+    json.dump({"sources": names, "sources_sha256": h.hexdigest(),
+               "workloads": {"w": {"dram_bytes_per_launch": 123, "profile": "p.md"}}},
+              open(fake / "profiles" / "traffic.json", "w"))
     monkeypatch.setattr(bench, "ROOT", str(fake))
-    got, src = bench.measured_traffic("mlra4_bf16_b16_h16_l4096_contig")
-    assert isinstance(got, int), src
+    assert bench.measured_traffic("w") == (123, "p.md")
     got, src = bench.measured_traffic("no_such_workload")
     assert got is None and "no ncu capture" in src
     with open(csrc / names[0], "a") as f:
         f.write("\n// edited\n")
-    got, src = bench.measured_traffic("mlra4_bf16_b16_h16_l4096_contig")
+    got, src = bench.measured_traffic("w")
     assert got is None and "changed" in src
