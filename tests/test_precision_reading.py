@@ -1,0 +1,86 @@
+"""The operand-precision reading, checked on the CPU against the fp64 oracle.
+
+The bf16 bound (max|err| <= 5e-3 max|ref|, mean|err| <= 5e-4 mean|ref|) fixes no
+operand type.  The kernels round the absorbed query (fp32) to bf16 hi + lo halves
+and the probabilities to bf16 hi + lo halves (head-rows and MLA kernels) or to
+fp16 (128-head kernel); everything else accumulates in fp32.  This emulation
+rounds the operands that way, computes the rest in fp64, and compares the
+decode output with the unabsorbed fp64 oracle on the workloads' own inputs:
+the roundings the kernels use stay inside the bound, and the cheaper ones they
+do not use (a single bf16 query, single bf16 probabilities) fall outside it on
+the workloads whose queries are N(0, 1).  It tests the choice, not the CUDA path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import mlra_oracle
+import workloads as W
+
+BF16_MAX, BF16_MEAN = 5e-3, 5e-4
+
+
+def _bf16(x):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).double().numpy()
+
+
+def _round(x, mode):
+    x = np.asarray(x, np.float64)
+    if mode == "hilo":
+        hi = _bf16(x)
+        return hi + _bf16(x - hi)
+    if mode == "bf16":
+        return _bf16(x)
+    if mode == "fp16":
+        return np.asarray(x, np.float32).astype(np.float16).astype(np.float64)
+    raise ValueError(mode)
+
+
+def _f32(x):
+    return np.asarray(x, np.float64).astype(np.float32).astype(np.float64)
+
+
+def _emulated(spec, inp, s, qmode, pmode):
+    """One sequence's decode output with the kernels' operand roundings."""
+    rows = W.sequence_cache(inp, s).double().numpy()
+    c, kr = mlra_oracle.split_cache_rows(rows, spec.n_blocks, spec.d_cb)
+    q_abs = _f32(oracle.absorb_query(inp.q_nope[s], inp.w_uk))   # the absorb kernel's fp32
+    qa = _round(q_abs, qmode)
+    q_rope = inp.q_rope[s].double().numpy()
+    w_uv = inp.w_uv.double().numpy()
+    h = q_abs.shape[0]
+    out = np.zeros((h, spec.d_h))
+    for hh in range(h):
+        for b in range(spec.n_blocks):
+            z = _f32((c[:, b] @ qa[hh, b] + kr @ q_rope[hh]) * spec.softmax_scale)
+            p = _f32(np.exp(z - z.max()))
+            o = (_round(p, pmode) @ c[:, b]) / p.sum()
+            out[hh] += o @ w_uv[b, hh]
+    return spec.branch_scale * out
+
+
+def _errors(name, qmode, pmode, L=2048, heads=16):
+    spec = W.scaled_down(W.WORKLOADS[name], 1, seqlen=L, n_heads=heads, seed=5)
+    inp = W.make_inputs(spec, "cpu")
+    ref = oracle.decode_batch(inp)[0].out
+    got = _emulated(spec, inp, 0, qmode, pmode)
+    e = np.abs(got - ref)
+    return e.max() / np.abs(ref).max(), e.mean() / np.abs(ref).mean()
+
+
+@pytest.mark.parametrize("name", ["mlra4_bf16_b8_h128_l131072_paged",
+                                  "mla_bf16_b8_h128_l131072_paged"])
+def test_kernel_roundings_are_inside_the_bound(name):
+    for pmode in ("hilo", "fp16"):
+        mx, mn = _errors(name, "hilo", pmode)
+        assert mx <= BF16_MAX / 3 and mn <= BF16_MEAN / 2, (pmode, mx, mn)
+
+
+@pytest.mark.parametrize("name", ["mlra4_bf16_b8_h128_l131072_paged",
+                                  "mla_bf16_b8_h128_l131072_paged"])
+def test_cheaper_roundings_are_outside_the_bound(name):
+    _, mn_q = _errors(name, "bf16", "hilo")     # a single bf16 query
+    _, mn_p = _errors(name, "hilo", "bf16")     # single bf16 probabilities
+    assert mn_q > BF16_MEAN and mn_p > BF16_MEAN, (mn_q, mn_p)
