@@ -80,3 +80,37 @@ def test_no_cpu_path():
     with pytest.raises(ValueError):
         mlra.absorb_q(cfg, torch.zeros(1, 16, 128, dtype=torch.bfloat16),
                       torch.zeros(4, 16, 128, 128, dtype=torch.bfloat16))
+
+
+def test_decode_step_validation_without_device(L):
+    """mlra_decode_step rejects bad arguments before it touches the device or the
+    workspace (a dummy, never dereferenced address stands in for it)."""
+    cfg = mlra.make_config(4, 128, 64, 16, 128)
+    ws = ctypes.c_void_p(256)
+
+    def call(batch, host_io, workspace):
+        return L.mlra_decode_step(ctypes.byref(cfg), None, None, None, batch, None, None, None,
+                                  0, None, 1, None, host_io, workspace, 1 << 20, None)
+
+    assert call(1, 2, ws) == 1                      # host_io neither 0 nor 1
+    assert call(-1, 0, ws) == 1                     # negative batch
+    assert call(1, 0, None) == 1                    # no workspace
+    assert call(1, 0, ctypes.c_void_p(16)) == 4     # workspace not 256-byte aligned
+    assert call(0, 1, ws) == 0                      # empty batch: nothing is launched
+    assert call(1, 0, ws) == 1                      # null inputs
+    assert L.mlra_decode_step(None, None, None, None, 1, None, None, None, 0, None, 1, None, 0,
+                              ws, 1 << 20, None) == 1
+
+
+def test_no_device_no_result(L):
+    """Without a usable GPU the library computes nothing on the host: a call that
+    needs the device reports MLRA_ERR_NO_DEVICE (after its argument checks)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    cfg = mlra.make_config(4, 128, 64, 16, 128)
+    sz = ctypes.c_size_t(0)
+    assert L.mlra_workspace_size(ctypes.byref(cfg), 4, None) == 1
+    assert L.mlra_step_workspace_size(None, 4, ctypes.byref(sz)) == 1
+    assert L.mlra_workspace_size(ctypes.byref(cfg), 4, ctypes.byref(sz)) == 8
+    assert L.mlra_step_workspace_size(ctypes.byref(cfg), 4, ctypes.byref(sz)) == 8
