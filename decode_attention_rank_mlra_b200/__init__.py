@@ -137,13 +137,22 @@ def _stream(stream) -> int:
     return stream.cuda_stream
 
 
-def _need(t: torch.Tensor, name: str, dtype: Optional[torch.dtype] = None):
+def _need(t: torch.Tensor, name: str, dtype: Optional[torch.dtype] = None, shape=None):
+    """A contiguous CUDA tensor on the current device (the library launches there),
+    of ``dtype`` and, when given, of ``shape`` (-1 matches any extent)."""
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None:
+        shape = tuple(int(x) for x in shape)
+        if t.dim() != len(shape) or any(w != -1 and w != g for w, g in zip(shape, t.shape)):
+            raise ValueError(f"{name} must have shape {shape} (-1: any), got {tuple(t.shape)}")
 
 
 def _check(fn: str, status: int):
@@ -154,13 +163,13 @@ def _check(fn: str, status: int):
 def absorb_q(cfg: Config, q_nope: torch.Tensor, w_uk: torch.Tensor,
              q_abs: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Step 1: q_abs[s,h,b,i] = sum_j W_uk[b,h,i,j] q_nope[s,h,j] (fp32 out)."""
-    _need(q_nope, "q_nope", cfg.torch_dtype)
-    _need(w_uk, "w_uk", cfg.torch_dtype)
+    _need(q_nope, "q_nope", cfg.torch_dtype, (-1, cfg.n_heads, cfg.d_h))
+    _need(w_uk, "w_uk", cfg.torch_dtype, (cfg.n_blocks, cfg.n_heads, cfg.d_cb, cfg.d_h))
     B = q_nope.shape[0]
     if q_abs is None:
         q_abs = torch.empty((B, cfg.n_heads, cfg.n_blocks, cfg.d_cb), dtype=torch.float32,
                             device=q_nope.device)
-    _need(q_abs, "q_abs", torch.float32)
+    _need(q_abs, "q_abs", torch.float32, (B, cfg.n_heads, cfg.n_blocks, cfg.d_cb))
     _check("mlra_absorb_q", lib().mlra_absorb_q(ctypes.byref(cfg), _ptr(q_nope), _ptr(w_uk),
                                                 _ptr(q_abs), B, _stream(stream)))
     return q_abs
@@ -178,6 +187,20 @@ def alloc_workspace(cfg: Config, batch: int, device=None) -> torch.Tensor:
     return _aligned_bytes(workspace_size(cfg, batch), device)
 
 
+def _attn_inputs(cfg: Config, q_abs, q_rope, kv_cache, page_table, seqlens, max_pages) -> int:
+    """Checks shared by the attention calls; returns the batch."""
+    _need(seqlens, "seqlens", torch.int32, (-1,))
+    B = seqlens.shape[0]
+    _need(q_abs, "q_abs", torch.float32, (B, cfg.n_heads, cfg.n_blocks, cfg.d_cb))
+    _need(q_rope, "q_rope", cfg.torch_dtype, (B, cfg.n_heads, cfg.d_r))
+    if page_table is not None:
+        _need(page_table, "page_table", torch.int32, (B, max_pages))
+        _need(kv_cache, "kv_cache", cfg.torch_dtype, (-1, cfg.page_size, cfg.D))
+    else:
+        _need(kv_cache, "kv_cache", cfg.torch_dtype, (B, max_pages, cfg.D))
+    return B
+
+
 def decode_attn(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor, kv_cache: torch.Tensor,
                 page_table: Optional[torch.Tensor], seqlens: torch.Tensor, max_pages: int,
                 workspace: torch.Tensor, stream=None) -> None:
@@ -186,16 +209,9 @@ def decode_attn(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor, kv_cache
     Paged: kv_cache [num_pages, 64, D], page_table [B, max_pages] int32.
     Contiguous: page_table None, kv_cache [B, max_len, D], max_pages = max_len.
     """
-    _need(q_abs, "q_abs", torch.float32)
-    _need(q_rope, "q_rope", cfg.torch_dtype)
-    _need(kv_cache, "kv_cache", cfg.torch_dtype)
-    _need(seqlens, "seqlens", torch.int32)
+    B = _attn_inputs(cfg, q_abs, q_rope, kv_cache, page_table, seqlens, max_pages)
     _need(workspace, "workspace", torch.uint8)
-    num_pages = 0
-    if page_table is not None:
-        _need(page_table, "page_table", torch.int32)
-        num_pages = kv_cache.shape[0]
-    B = seqlens.shape[0]
+    num_pages = kv_cache.shape[0] if page_table is not None else 0
     _check("mlra_decode_attn", lib().mlra_decode_attn(
         ctypes.byref(cfg), _ptr(q_abs), _ptr(q_rope), _ptr(kv_cache), num_pages, _ptr(page_table),
         int(max_pages), _ptr(seqlens), B, _ptr(workspace), workspace.numel(), _stream(stream)))
@@ -211,8 +227,9 @@ def splitkv_combine(cfg: Config, workspace: torch.Tensor, batch: int,
                                device=dev)
     if lse is None:
         lse = torch.empty((batch, cfg.n_heads, cfg.n_blocks), dtype=torch.float32, device=dev)
-    _need(o_latent, "o_latent", torch.float32)
-    _need(lse, "lse", torch.float32)
+    _need(workspace, "workspace", torch.uint8)
+    _need(o_latent, "o_latent", torch.float32, (batch, cfg.n_heads, cfg.n_blocks, cfg.d_cb))
+    _need(lse, "lse", torch.float32, (batch, cfg.n_heads, cfg.n_blocks))
     _check("mlra_splitkv_combine", lib().mlra_splitkv_combine(
         ctypes.byref(cfg), _ptr(workspace), workspace.numel(), batch, _ptr(o_latent), _ptr(lse),
         _stream(stream)))
@@ -222,12 +239,12 @@ def splitkv_combine(cfg: Config, workspace: torch.Tensor, batch: int,
 def out_proj(cfg: Config, o_latent: torch.Tensor, w_uv: torch.Tensor,
              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Step 3: out[s,h,:] = branch_scale * sum_b W_uv[b,h]^T o_latent[s,h,b] (fp32)."""
-    _need(o_latent, "o_latent", torch.float32)
-    _need(w_uv, "w_uv", cfg.torch_dtype)
+    _need(o_latent, "o_latent", torch.float32, (-1, cfg.n_heads, cfg.n_blocks, cfg.d_cb))
+    _need(w_uv, "w_uv", cfg.torch_dtype, (cfg.n_blocks, cfg.n_heads, cfg.d_cb, cfg.d_h))
     B = o_latent.shape[0]
     if out is None:
         out = torch.empty((B, cfg.n_heads, cfg.d_h), dtype=torch.float32, device=o_latent.device)
-    _need(out, "out", torch.float32)
+    _need(out, "out", torch.float32, (B, cfg.n_heads, cfg.d_h))
     _check("mlra_out_proj", lib().mlra_out_proj(ctypes.byref(cfg), _ptr(o_latent), _ptr(w_uv),
                                                 _ptr(out), B, _stream(stream)))
     return out
@@ -241,15 +258,16 @@ def combine_out_proj(cfg: Config, workspace: torch.Tensor, batch: int, w_uv: tor
     ``o_latent`` / ``lse`` are written when given (needed when the fused
     tensor-core kernel does not apply).
     """
-    _need(w_uv, "w_uv", cfg.torch_dtype)
+    _need(workspace, "workspace", torch.uint8)
+    _need(w_uv, "w_uv", cfg.torch_dtype, (cfg.n_blocks, cfg.n_heads, cfg.d_cb, cfg.d_h))
     if out is None:
         out = torch.empty((batch, cfg.n_heads, cfg.d_h), dtype=torch.float32,
                           device=workspace.device)
-    _need(out, "out", torch.float32)
+    _need(out, "out", torch.float32, (batch, cfg.n_heads, cfg.d_h))
     if o_latent is not None:
-        _need(o_latent, "o_latent", torch.float32)
+        _need(o_latent, "o_latent", torch.float32, (batch, cfg.n_heads, cfg.n_blocks, cfg.d_cb))
     if lse is not None:
-        _need(lse, "lse", torch.float32)
+        _need(lse, "lse", torch.float32, (batch, cfg.n_heads, cfg.n_blocks))
     _check("mlra_combine_out_proj", lib().mlra_combine_out_proj(
         ctypes.byref(cfg), _ptr(workspace), workspace.numel(), batch, _ptr(w_uv), _ptr(out),
         _ptr(o_latent), _ptr(lse), _stream(stream)))
@@ -263,18 +281,20 @@ def cache_append(cfg: Config, c_new: torch.Tensor, k_rope_new: torch.Tensor,
                  device_status: Optional[torch.Tensor] = None, stream=None) -> None:
     """Cache write: each sequence's new row (per-block RMSNorm x gain x alpha_kv,
     rotated RoPE key) at token ``positions[s]``, in place in ``kv_cache``."""
-    _need(c_new, "c_new", cfg.torch_dtype)
-    _need(k_rope_new, "k_rope_new", cfg.torch_dtype)
-    _need(rms_gamma, "rms_gamma", torch.float32)
-    _need(kv_cache, "kv_cache", cfg.torch_dtype)
-    _need(positions, "positions", torch.int32)
+    _need(positions, "positions", torch.int32, (-1,))
+    B = positions.shape[0]
+    _need(c_new, "c_new", cfg.torch_dtype, (B, cfg.n_blocks * cfg.d_cb))
+    _need(k_rope_new, "k_rope_new", cfg.torch_dtype, (B, cfg.d_r))
+    _need(rms_gamma, "rms_gamma", torch.float32, (cfg.n_blocks * cfg.d_cb,))
     num_pages = 0
     if page_table is not None:
-        _need(page_table, "page_table", torch.int32)
+        _need(page_table, "page_table", torch.int32, (B, max_pages))
+        _need(kv_cache, "kv_cache", cfg.torch_dtype, (-1, cfg.page_size, cfg.D))
         num_pages = kv_cache.shape[0]
+    else:
+        _need(kv_cache, "kv_cache", cfg.torch_dtype, (B, max_pages, cfg.D))
     if device_status is not None:
-        _need(device_status, "device_status", torch.int32)
-    B = positions.shape[0]
+        _need(device_status, "device_status", torch.int32, (-1,))
     _check("mlra_cache_append", lib().mlra_cache_append(
         ctypes.byref(cfg), _ptr(c_new), _ptr(k_rope_new), _ptr(rms_gamma), float(alpha_kv),
         float(rms_eps), float(rope_theta), _ptr(kv_cache), num_pages, _ptr(page_table),
@@ -329,14 +349,16 @@ def decode_step(cfg: Config, q_nope: torch.Tensor, q_rope: torch.Tensor, seqlens
     if q_nope.shape != (B, h, cfg.d_h) or q_rope.shape != (B, h, cfg.d_r) \
             or out.shape != (B, h, cfg.d_h):
         raise ValueError("q_nope / q_rope / out shapes do not match seqlens and cfg")
-    _need(w_uk, "w_uk", cfg.torch_dtype)
-    _need(w_uv, "w_uv", cfg.torch_dtype)
-    _need(kv_cache, "kv_cache", cfg.torch_dtype)
+    _need(w_uk, "w_uk", cfg.torch_dtype, (cfg.n_blocks, cfg.n_heads, cfg.d_cb, cfg.d_h))
+    _need(w_uv, "w_uv", cfg.torch_dtype, (cfg.n_blocks, cfg.n_heads, cfg.d_cb, cfg.d_h))
     _need(workspace, "workspace", torch.uint8)
     num_pages = 0
     if page_table is not None:
-        _need(page_table, "page_table", torch.int32)
+        _need(page_table, "page_table", torch.int32, (B, max_pages))
+        _need(kv_cache, "kv_cache", cfg.torch_dtype, (-1, cfg.page_size, cfg.D))
         num_pages = kv_cache.shape[0]
+    else:
+        _need(kv_cache, "kv_cache", cfg.torch_dtype, (B, max_pages, cfg.D))
     _check("mlra_decode_step", lib().mlra_decode_step(
         ctypes.byref(cfg), _ptr(q_nope), _ptr(q_rope), _ptr(seqlens), B, _ptr(w_uk), _ptr(w_uv),
         _ptr(kv_cache), num_pages, _ptr(page_table), int(max_pages), _ptr(out), int(on_host),
@@ -359,20 +381,15 @@ def decode_attn_noalloc(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor,
     ``splitkv_combine``; ``device_status`` (one int32 on the device) receives
     the call's device error word.
     """
-    _need(q_abs, "q_abs", torch.float32)
-    _need(q_rope, "q_rope", cfg.torch_dtype)
-    _need(kv_cache, "kv_cache", cfg.torch_dtype)
-    _need(seqlens, "seqlens", torch.int32)
-    _need(o_latent, "o_latent", torch.float32)
+    B = _attn_inputs(cfg, q_abs, q_rope, kv_cache, page_table, seqlens, max_pages)
+    _need(o_latent, "o_latent", torch.float32, (B, cfg.n_heads, cfg.n_blocks, cfg.d_cb))
     if lse is not None:
-        _need(lse, "lse", torch.float32)
+        _need(lse, "lse", torch.float32, (B, cfg.n_heads, cfg.n_blocks))
     if device_status is not None:
-        _need(device_status, "device_status", torch.int32)
-    num_pages = 0
-    if page_table is not None:
-        _need(page_table, "page_table", torch.int32)
-        num_pages = kv_cache.shape[0]
-    B = seqlens.shape[0]
+        _need(device_status, "device_status", torch.int32, (-1,))
+        if device_status.numel() < 1:
+            raise ValueError("device_status must hold at least one int32")
+    num_pages = kv_cache.shape[0] if page_table is not None else 0
     _check("mlra_decode_attn_noalloc", lib().mlra_decode_attn_noalloc(
         ctypes.byref(cfg), _ptr(q_abs), _ptr(q_rope), _ptr(kv_cache), num_pages, _ptr(page_table),
         int(max_pages), _ptr(seqlens), B, _ptr(o_latent), _ptr(lse), _ptr(device_status),

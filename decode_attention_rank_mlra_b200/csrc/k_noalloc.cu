@@ -20,26 +20,53 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 
 // Device-side scratch shared by every call of mlra_decode_attn_noalloc.  In
 // host code this name is only a stand-in: its device address comes from
-// cudaGetSymbolAddress (once per device, below).
+// cudaGetSymbolAddress (once per device and context, below).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDev = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDev] = {nullptr};
+struct ScratchAddr {
+  void* ctx;  // the context the address was looked up in
+  void* ptr;
+};
+ScratchAddr g_scratch[kMaxDev] = {};
 
-// Device address of the scratch on the current device; looked up on the first
-// call made with that device current.
+// The current context (CUcontext) through the driver entry point, or NULL.
+void* current_context() {
+  using GetCurrent = int (*)(void**);
+  static GetCurrent fn = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCurrent>(p);
+    looked = true;
+  }
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of the scratch on the current device.  Looked up with that
+// device current on the first call, and again whenever the device's context
+// has changed since (a cudaDeviceReset destroys the context and the module
+// that holds the array; the next context loads it again, possibly elsewhere).
 mlra_status_t scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return MLRA_ERR_NO_DEVICE;
+  // (no context may be current yet in this thread: then it is looked up, which
+  // also makes the device's primary context current)
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch[dev].ptr || ctx == nullptr || g_scratch[dev].ctx != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return MLRA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    g_scratch[dev] = ScratchAddr{current_context(), p};
   }
-  *out = g_scratch_ptr[dev];
+  *out = g_scratch[dev].ptr;
   return MLRA_OK;
 }
 

@@ -52,29 +52,20 @@ mlra_status_t check_cfg(const mlra_config_t* c) {
   return MLRA_OK;
 }
 
-// 1 = tensor core, 2 = SIMT, 0 = unsupported.  MLRA_DECODE_KERNEL=simt forces
-// the SIMT kernel (used by tests to cross-check the two paths).
+// 1 = tensor core, 2 = SIMT, 0 = unsupported.  The fp32 cache and the bf16
+// shapes the tensor-core kernels do not take (head counts other than 16, 32,
+// 64 or multiples of 128; latent blocks other than 128, or 512 for one block)
+// run on the fp32 SIMT kernel.
 int choose_kernel(const mlra_config_t& c, int dev) {
-  static int forced = -1;
-  if (forced < 0) {
-    const char* e = getenv("MLRA_DECODE_KERNEL");
-    forced = (e && strcmp(e, "simt") == 0) ? 2 : 0;
-  }
-  if (forced == 2) return simt_supported(c) ? 2 : 0;
   if (c.dtype == MLRA_BF16 && device_is_sm100(dev) && tc_supported(c)) return 1;
   if (simt_supported(c)) return 2;
   return 0;
 }
 
 // Tensor-core absorption / output projection on this device for this config?
-// MLRA_PROJ_KERNEL=simt forces the SIMT kernels (tests cross-check both).
+// (bf16 with d_h = 128; the SIMT kernels take the rest.)
 bool use_proj_tc(const mlra_config_t& c) {
-  static int forced = -1;
-  if (forced < 0) {
-    const char* e = getenv("MLRA_PROJ_KERNEL");
-    forced = (e && strcmp(e, "simt") == 0) ? 1 : 0;
-  }
-  if (forced == 1 || !proj_tc_supported(c)) return false;
+  if (!proj_tc_supported(c)) return false;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   return device_is_sm100(dev);

@@ -295,8 +295,9 @@ MLRA_API mlra_status_t mlra_get_device_error(const void* workspace, size_t works
  *                   MLRA_ERR_TIMEOUT, MLRA_ERR_INVALID_ARG for clamped seqlens)
  * Returns MLRA_ERR_WORKSPACE, launching nothing, when the scratch this batch
  * needs (mlra_workspace_size) exceeds 16 MiB.  The first call on a device looks
- * up the array's device address with that device current; make that first
- * call before capturing any stream.  All calls share the one array and it
+ * up the array's device address with that device current (and again after the
+ * device's context changed, e.g. after cudaDeviceReset); make that first call
+ * before capturing any stream.  All calls share the one array and it
  * keeps the last call's contents: calls ordered on one stream are safe, calls
  * that overlap on the GPU (other streams, other host threads) race on it.
  */

@@ -17,6 +17,13 @@ import workloads as W
 F32_MAX_REL = 1e-5
 BF16_MAX = 5e-3
 BF16_MEAN = 5e-4
+# fp32 elementwise error with a floor of 1e-3 * max|ref| (reported beside the
+# normwise figure).  Plain fp32 arithmetic of the same computation already
+# reaches ~3e-5 there (tests/test_precision_reading.py), so 1e-5 elementwise is
+# out of reach of any fp32 kernel; the bound asserted is 1e-3, which any result
+# meeting the normwise bound with errors spread like rounding noise meets.
+F32_ELEM_FLOOR = 1e-3
+F32_ELEM_TOL = 1e-3
 
 
 def config_of(spec: W.WorkloadSpec) -> mlra.Config:
@@ -48,9 +55,13 @@ def check_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = "out")
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     err = np.abs(got - ref)
     if dtype == "f32":
-        rel = err.max() / max(np.abs(ref).max(), 1e-30)
+        rmax = max(np.abs(ref).max(), 1e-30)
+        rel = err.max() / rmax
         assert rel <= F32_MAX_REL, f"{what}: max rel err {rel:.3e} > {F32_MAX_REL}"
-        return dict(max_rel=rel)
+        elem = (err / np.maximum(np.abs(ref), F32_ELEM_FLOOR * rmax)).max()
+        assert elem <= F32_ELEM_TOL, f"{what}: elementwise err {elem:.3e} > {F32_ELEM_TOL}"
+        print(f"{what}: fp32 normwise {rel:.3e}, elementwise (floor 1e-3 max|ref|) {elem:.3e}")
+        return dict(max_rel=rel, elem_rel=elem)
     mx = err.max() / max(np.abs(ref).max(), 1e-30)
     mn = err.mean() / max(np.abs(ref).mean(), 1e-30)
     assert mx <= BF16_MAX, f"{what}: max err {mx:.3e} * max|ref| > {BF16_MAX}"
@@ -73,38 +84,55 @@ def compare_batch(inp: W.DecodeInputs, got: Dict[str, torch.Tensor],
     check_close(lat_got, lat_ref, spec.dtype, "o_lat")
     lse_ref = np.stack([r.lse[hs] for r in refs])
     lse_got = got["lse"].double().numpy()[seqs][:, hs]
-    finite = np.isfinite(lse_ref)
-    assert np.array_equal(finite, np.isfinite(lse_got))
-    if finite.any():
-        d = np.abs(lse_got[finite] - lse_ref[finite])
-        if spec.dtype == "f32":
-            tol = 1e-5 * (1.0 + np.abs(lse_ref[finite]))
-        else:
-            # A logit reaches the softmax with an error of about 2^-15 of
-            # scale * sum_j |q_j k_j| (bf16 hi + lo queries, fp32 accumulation
-            # over 192 or 576 products), which can exceed |logit| many times
-            # over when the products cancel; the lse inherits it.
-            tol = 2e-3 + 2.0 ** -15 * logit_magnitude(inp, seqs, hs)[finite]
-        worst = int(np.argmax(d - tol))
-        assert np.all(d <= tol), f"lse err {d[worst]:.3e} > tol {tol[worst]:.3e}"
+    mag = None if spec.dtype == "f32" else logit_magnitude(inp, seqs, hs)
+    check_lse(lse_got, lse_ref, spec.dtype, mag)
     return stats
 
 
 def logit_magnitude(inp: W.DecodeInputs, seqs: Sequence[int], heads: Sequence[int]) -> np.ndarray:
     """[seq, head, branch] max over tokens of scale * sum_j |q_j k_j| (latent + RoPE)."""
-    from oracle.mlra_oracle import split_cache_rows
     spec = inp.spec
-    nb = spec.n_blocks
-    out = np.zeros((len(seqs), len(heads), nb))
+    out = np.zeros((len(seqs), len(heads), spec.n_blocks))
     for i, s in enumerate(seqs):
         rows = W.sequence_cache(inp, s)
-        if rows.shape[0] == 0:
-            continue
-        c, kr = split_cache_rows(rows.cpu(), nb, spec.d_cb)    # [L, nb, d_cb], [L, d_r]
-        qa = np.abs(oracle.absorb_query(inp.q_nope[s].cpu(), inp.w_uk.cpu()))  # [H, nb, d_cb]
-        qr = np.abs(inp.q_rope[s].cpu().double().numpy())      # [H, d_r]
-        rope = qr[heads] @ np.abs(kr).T                        # [h, L]
-        for b in range(nb):
-            lat = qa[heads, b] @ np.abs(c[:, b]).T             # [h, L]
-            out[i, :, b] = spec.softmax_scale * np.max(lat + rope, axis=1)
+        out[i] = rows_logit_magnitude(spec, rows.cpu(), inp.q_nope[s].cpu(), inp.q_rope[s].cpu(),
+                                      inp.w_uk.cpu(), heads)
     return out
+
+
+def rows_logit_magnitude(spec, rows, q_nope_s, q_rope_s, w_uk, heads) -> np.ndarray:
+    """[head, branch] max over one sequence's cache rows of scale * sum_j |q_j k_j|."""
+    from oracle.mlra_oracle import split_cache_rows
+    nb = spec.n_blocks
+    out = np.zeros((len(heads), nb))
+    if rows.shape[0] == 0:
+        return out
+    c, kr = split_cache_rows(rows, nb, spec.d_cb)              # [L, nb, d_cb], [L, d_r]
+    qa = np.abs(oracle.absorb_query(q_nope_s, w_uk))           # [H, nb, d_cb]
+    qr = np.abs(np.asarray(q_rope_s.double().numpy() if hasattr(q_rope_s, "double") else q_rope_s))
+    rope = qr[heads] @ np.abs(kr).T                            # [h, L]
+    for b in range(nb):
+        lat = qa[heads, b] @ np.abs(c[:, b]).T                 # [h, L]
+        out[:, b] = spec.softmax_scale * np.max(lat + rope, axis=1)
+    return out
+
+
+def check_lse(got_lse: np.ndarray, ref_lse: np.ndarray, dtype: str, magnitude=None):
+    """lse against the oracle: fp32 to 1e-5 (1 + |lse|); bf16 to 2e-3 plus
+    2^-15 of the logit magnitude (a logit reaches the softmax with an error of
+    about 2^-15 of scale * sum_j |q_j k_j|: bf16 hi + lo queries, fp32
+    accumulation over 192 or 576 products, which can exceed |logit| many times
+    over when the products cancel; the lse inherits it)."""
+    got_lse = np.asarray(got_lse, np.float64)
+    ref_lse = np.asarray(ref_lse, np.float64)
+    finite = np.isfinite(ref_lse)
+    assert np.array_equal(finite, np.isfinite(got_lse))
+    if not finite.any():
+        return
+    d = np.abs(got_lse[finite] - ref_lse[finite])
+    if dtype == "f32":
+        tol = 1e-5 * (1.0 + np.abs(ref_lse[finite]))
+    else:
+        tol = 2e-3 + 2.0 ** -15 * np.asarray(magnitude)[finite]
+    worst = int(np.argmax(d - tol))
+    assert np.all(d <= tol), f"lse err {d[worst]:.3e} > tol {tol[worst]:.3e}"

@@ -78,31 +78,93 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
 
 
 def test_traffic_only_for_the_captured_kernel_sources(tmp_path, monkeypatch):
-    """roofline.traffic comes from an ncu capture only while the attention
-    kernels' sources hash to the captured ones: a tree whose capture matches
-    gives the figure, an unknown workload none, an edited source none."""
+    """roofline.traffic comes from an ncu capture only while the sources of the
+    kernel it was measured on hash to the captured ones: a matching entry gives
+    the figure, an unknown workload none, an edited source none (for the
+    workloads that depend on it only)."""
     import hashlib
     import json
     import shutil
 
     import bench
-    names = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["sources"]
     fake = tmp_path / "root"
     (fake / "profiles").mkdir(parents=True)
     csrc = fake / "decode_attention_rank_mlra_b200" / "csrc"
     csrc.mkdir(parents=True)
-    h = hashlib.sha256()
+    names = ["k_decode_tc.cu", "k_decode_wide.cu", "tc_common.cuh"]
     for n in names:
         shutil.copy(os.path.join(ROOT, "decode_attention_rank_mlra_b200", "csrc", n), csrc)
-        h.update((csrc / n).read_bytes())
-    json.dump({"sources": names, "sources_sha256": h.hexdigest(),
-               "workloads": {"w": {"dram_bytes_per_launch": 123, "profile": "p.md"}}},
-              open(fake / "profiles" / "traffic.json", "w"))
+
+    def sha(files):
+        h = hashlib.sha256()
+        for n in files:
+            h.update((csrc / n).read_bytes())
+        return h.hexdigest()
+
+    a_src, b_src = ["k_decode_tc.cu", "tc_common.cuh"], ["k_decode_wide.cu", "tc_common.cuh"]
+    json.dump({"workloads": {
+        "a": {"dram_bytes_per_launch": 123, "profile": "p.md", "sources": a_src,
+              "sources_sha256": sha(a_src)},
+        "b": {"dram_bytes_per_launch": 456, "profile": "q.md", "sources": b_src,
+              "sources_sha256": sha(b_src)}}},
+        open(fake / "profiles" / "traffic.json", "w"))
     monkeypatch.setattr(bench, "ROOT", str(fake))
-    assert bench.measured_traffic("w") == (123, "p.md")
+    assert bench.measured_traffic("a") == (123, "p.md")
+    assert bench.measured_traffic("b") == (456, "q.md")
     got, src = bench.measured_traffic("no_such_workload")
     assert got is None and "no ncu capture" in src
-    with open(csrc / names[0], "a") as f:
+    with open(csrc / "k_decode_tc.cu", "a") as f:
         f.write("\n// edited\n")
-    got, src = bench.measured_traffic("w")
+    got, src = bench.measured_traffic("a")
     assert got is None and "changed" in src
+    assert bench.measured_traffic("b") == (456, "q.md")
+
+
+def test_committed_traffic_entries_name_their_kernel_sources():
+    """Every committed entry lists the files its figure depends on."""
+    import json
+    t = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for w, e in t["workloads"].items():
+        assert e["sources"] and len(e["sources_sha256"]) == 64, w
+        for n in e["sources"]:
+            assert os.path.exists(os.path.join(ROOT, "decode_attention_rank_mlra_b200", "csrc", n))
+
+
+def test_both_arms_print_the_same_config(monkeypatch):
+    """The reference arm's config object is the one our arm prints (built from
+    the workload alone, no device needed), for every workload."""
+    import bench
+    import workloads as W
+    for name in bench.PER_CONFIG:
+        spec = W.WORKLOADS[name]
+        c = bench.workload_config(spec, 1)
+        assert c["workload"] == name and c["cached_tokens"] == int(W.seqlens_for(spec).sum())
+        copies = bench.cache_copies(spec)
+        nbytes = bench.cache_elems(spec) * spec.elem_bytes
+        # rotating copies exceed three L2s, else one copy already does, else flush
+        assert (copies > 1 and copies * nbytes > 3 * bench.L2_BYTES) or \
+            (copies == 1 and nbytes > 3 * bench.L2_BYTES) or (copies == 0 and 8 * nbytes <= 3 * bench.L2_BYTES)
+        assert ("flushed" in c["l2"]) == (copies == 0)
+
+    class Args:
+        workload = "mlra4_f32_b1_h4_l256"
+        steps = 1
+        warmup = 0
+        impl = "reference"
+
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    res = bench.run_reference(Args())
+    assert res["config"] == bench.workload_config(W.WORKLOADS[Args.workload], 1)
+
+
+def test_default_headline_is_the_largest_workload():
+    import bench
+    import workloads as W
+    sizes = {n: int(W.seqlens_for(W.WORKLOADS[n]).sum()) * W.WORKLOADS[n].D
+             * W.WORKLOADS[n].elem_bytes for n in bench.PER_CONFIG}
+    assert bench.DEFAULT_WORKLOAD == max(sizes, key=sizes.get)
+    assert bench.parse([]).workload == bench.DEFAULT_WORKLOAD
+    assert bench.split_workloads("all", bench.DEFAULT_WORKLOAD) == [
+        n for n in bench.PER_CONFIG if n != bench.DEFAULT_WORKLOAD]
+    assert bench.split_workloads("none", bench.DEFAULT_WORKLOAD) == []

@@ -12,7 +12,8 @@ import torch
 import decode_attention_rank_mlra_b200 as mlra
 import oracle
 import workloads as W
-from parity_util import check_close, compare_batch, config_of, run_gpu
+from parity_util import (check_close, check_lse, compare_batch, config_of, run_gpu,
+                         rows_logit_magnitude)
 
 pytestmark = pytest.mark.gpu
 
@@ -347,3 +348,8 @@ def test_full_size_sampled(name, samples):
                     f"{name} seq {seq}")
         check_close(got["o_lat"][seq, heads].double().numpy(), ref.o_lat[heads], spec.dtype,
                     f"{name} seq {seq} o_lat")
+        rows = W.token_rows(spec, seq, 0, int(L_all[seq]))
+        w_uk, _ = W.weights(spec)
+        q_nope, q_rope = W.queries(spec)
+        mag = rows_logit_magnitude(spec, rows, q_nope[seq], q_rope[seq], w_uk, heads)
+        check_lse(got["lse"][seq, heads].double().numpy(), ref.lse[heads], spec.dtype, mag)

@@ -312,3 +312,62 @@ def test_planted_mistake_is_caught(which, monkeypatch):
     out_bf, lse_bf = _brute_force(P)
     r = _oracle(P)
     assert not (np.allclose(r.out, out_bf, rtol=1e-9) and np.allclose(r.lse, lse_bf, rtol=1e-9))
+
+
+# ---- the oracle's input plumbing: cache-row split and sampled regeneration ----
+
+def test_split_cache_rows_takes_blocks_then_the_rope_key():
+    """A cache row is [c_0 | c_1 | ... | c_{nb-1} | k_rope] (4.5 d_h per token at
+    d_h = 128: Key Contributions #2).  Rows built from known blocks with
+    distinct integer values split back into exactly those blocks, the RoPE
+    key taken from offset nb * d_cb."""
+    L, nb, d_cb, d_r = 3, 4, 5, 2
+    c = np.arange(L * nb * d_cb, dtype=np.float64).reshape(L, nb, d_cb)
+    kr = -1.0 - np.arange(L * d_r, dtype=np.float64).reshape(L, d_r)
+    rows = np.concatenate([np.concatenate([c[t, b] for b in range(nb)] + [kr[t]])[None]
+                           for t in range(L)])
+    assert rows.shape == (L, nb * d_cb + d_r)
+    c2, kr2 = om.split_cache_rows(rows, nb, d_cb)
+    assert np.array_equal(c2, c) and np.array_equal(kr2, kr)
+    # block b of token t starts at column b * d_cb; the RoPE key at nb * d_cb
+    assert c2[2, 3, 0] == rows[2, 3 * d_cb] and kr2[1, 0] == rows[1, nb * d_cb]
+    # the cache-write oracle lays a row out the same way
+    g = np.ones(nb * d_cb)
+    new = oracle.cache_rows(c.reshape(L, -1), kr, g, nb, 1.0, 0.0, np.zeros(L), 10000.0)
+    c3, kr3 = om.split_cache_rows(new, nb, d_cb)
+    np.testing.assert_allclose(kr3, kr, rtol=0, atol=0)   # RoPE at position 0 is the identity
+    norm = c / np.sqrt(np.mean(c * c, axis=-1, keepdims=True))
+    np.testing.assert_allclose(c3, norm, rtol=1e-15)
+
+
+def test_split_cache_rows_same_latent_for_mla_and_mlra4():
+    """MLA (one block of 512 + 64) and MLRA-4 (4 x 128 + 64) read the same 576
+    columns: the latent part of a row is the same bytes either way."""
+    rng = np.random.default_rng(3)
+    rows = rng.standard_normal((7, 576))
+    c4, kr4 = om.split_cache_rows(rows, 4, 128)
+    c1, kr1 = om.split_cache_rows(rows, 1, 512)
+    assert np.array_equal(c4.reshape(7, 512), c1.reshape(7, 512))
+    assert np.array_equal(kr4, kr1) and kr4.shape == (7, 64)
+
+
+@pytest.mark.parametrize("name,seq,L", [
+    ("mlra4_bf16_b64_h32_l16384_paged", 2, 300),
+    ("mlra4_bf16_b128_h16_ragged1k_64k_paged", 1, 4100),
+    ("mla_bf16_b8_h128_l131072_paged", 0, 130),
+    ("mlra4_bf16_b16_h16_l4096_contig", 1, 70),
+])
+def test_decode_sampled_equals_decode_batch(name, seq, L):
+    """decode_sampled (one sequence's inputs redrawn from their seeds, used at
+    full sizes) gives exactly what decode_batch gives on the same sequence of
+    the whole generated batch (paged or contiguous, other sequences present)."""
+    import workloads as W
+    base = W.WORKLOADS[name]
+    heads = [0, base.n_heads - 1]
+    lens = np.array([L + 7 * s for s in range(seq + 2)], np.int32)
+    spec = W.scaled_down(base, len(lens), seqlen=int(lens.max()), seed=9)
+    inp = W.make_inputs(spec, "cpu", seqlens=lens)
+    whole = oracle.decode_batch(inp, heads=heads, seqs=[seq])[0]
+    one = oracle.decode_sampled(spec, seq, heads, int(lens[seq]))
+    for k in ("out", "lse", "o_lat", "v"):
+        assert np.array_equal(getattr(one, k)[heads], getattr(whole, k)[heads]), k
