@@ -38,7 +38,7 @@ EXPORTS = [
     "mlra_status_string", "mlra_version", "mlra_absorb_q", "mlra_workspace_size",
     "mlra_decode_attn", "mlra_splitkv_combine", "mlra_out_proj", "mlra_get_device_error",
     "mlra_decode_kernel_kind", "mlra_decode_attn_noalloc", "mlra_combine_out_proj",
-    "mlra_cache_append", "mlra_step_workspace_size", "mlra_decode_step",
+    "mlra_cache_append", "mlra_step_workspace_size", "mlra_decode_step", "mlra_absorb_q_rope",
 ]
 
 
@@ -96,6 +96,7 @@ def lib() -> ctypes.CDLL:
         "mlra_status_string": (ctypes.c_char_p, [I32]),
         "mlra_version": (I32, []),
         "mlra_absorb_q": (I32, [CP, P, P, P, I32, P]),
+        "mlra_absorb_q_rope": (I32, [CP, P, P, P, ctypes.c_float, ctypes.c_float, P, P, P, I32, P]),
         "mlra_workspace_size": (I32, [CP, I32, ctypes.POINTER(SZ)]),
         "mlra_decode_attn": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, SZ, P]),
         "mlra_splitkv_combine": (I32, [CP, P, SZ, I32, P, P, P]),
@@ -155,6 +156,15 @@ def _need(t: torch.Tensor, name: str, dtype: Optional[torch.dtype] = None, shape
             raise ValueError(f"{name} must have shape {shape} (-1: any), got {tuple(t.shape)}")
 
 
+def _contig_cache(kv_cache: torch.Tensor, cfg: Config, batch: int, max_len: int):
+    """A contiguous cache [>= batch, max_len, D]: row s * max_len + t is token t
+    of sequence s (a cache allocated for more sequences than the call's batch
+    is fine)."""
+    _need(kv_cache, "kv_cache", cfg.torch_dtype, (-1, max_len, cfg.D))
+    if kv_cache.shape[0] < batch:
+        raise ValueError(f"kv_cache holds {kv_cache.shape[0]} sequences, the batch is {batch}")
+
+
 def _check(fn: str, status: int):
     if status != 0:
         raise MlraError(fn, status)
@@ -173,6 +183,31 @@ def absorb_q(cfg: Config, q_nope: torch.Tensor, w_uk: torch.Tensor,
     _check("mlra_absorb_q", lib().mlra_absorb_q(ctypes.byref(cfg), _ptr(q_nope), _ptr(w_uk),
                                                 _ptr(q_abs), B, _stream(stream)))
     return q_abs
+
+
+def absorb_q_rope(cfg: Config, q_nope: torch.Tensor, q_rope: torch.Tensor,
+                  positions: torch.Tensor, alpha_q: float, w_uk: torch.Tensor,
+                  q_abs: Optional[torch.Tensor] = None, q_rope_out: Optional[torch.Tensor] = None,
+                  rope_theta: float = 10000.0, stream=None):
+    """Step 1 with the query-side calibration: q_abs = alpha_q W_uk q_nope (fp32)
+    and q_rope_out = RoPE(alpha_q q_rope) at ``positions[s]`` (storage dtype).
+    Returns (q_abs, q_rope_out)."""
+    _need(positions, "positions", torch.int32, (-1,))
+    B = positions.shape[0]
+    _need(q_nope, "q_nope", cfg.torch_dtype, (B, cfg.n_heads, cfg.d_h))
+    _need(q_rope, "q_rope", cfg.torch_dtype, (B, cfg.n_heads, cfg.d_r))
+    _need(w_uk, "w_uk", cfg.torch_dtype, (cfg.n_blocks, cfg.n_heads, cfg.d_cb, cfg.d_h))
+    if q_abs is None:
+        q_abs = torch.empty((B, cfg.n_heads, cfg.n_blocks, cfg.d_cb), dtype=torch.float32,
+                            device=q_nope.device)
+    if q_rope_out is None:
+        q_rope_out = torch.empty_like(q_rope)
+    _need(q_abs, "q_abs", torch.float32, (B, cfg.n_heads, cfg.n_blocks, cfg.d_cb))
+    _need(q_rope_out, "q_rope_out", cfg.torch_dtype, (B, cfg.n_heads, cfg.d_r))
+    _check("mlra_absorb_q_rope", lib().mlra_absorb_q_rope(
+        ctypes.byref(cfg), _ptr(q_nope), _ptr(q_rope), _ptr(positions), float(alpha_q),
+        float(rope_theta), _ptr(w_uk), _ptr(q_abs), _ptr(q_rope_out), B, _stream(stream)))
+    return q_abs, q_rope_out
 
 
 def workspace_size(cfg: Config, batch: int) -> int:
@@ -197,7 +232,7 @@ def _attn_inputs(cfg: Config, q_abs, q_rope, kv_cache, page_table, seqlens, max_
         _need(page_table, "page_table", torch.int32, (B, max_pages))
         _need(kv_cache, "kv_cache", cfg.torch_dtype, (-1, cfg.page_size, cfg.D))
     else:
-        _need(kv_cache, "kv_cache", cfg.torch_dtype, (B, max_pages, cfg.D))
+        _contig_cache(kv_cache, cfg, B, max_pages)
     return B
 
 
@@ -292,7 +327,7 @@ def cache_append(cfg: Config, c_new: torch.Tensor, k_rope_new: torch.Tensor,
         _need(kv_cache, "kv_cache", cfg.torch_dtype, (-1, cfg.page_size, cfg.D))
         num_pages = kv_cache.shape[0]
     else:
-        _need(kv_cache, "kv_cache", cfg.torch_dtype, (B, max_pages, cfg.D))
+        _contig_cache(kv_cache, cfg, B, max_pages)
     if device_status is not None:
         _need(device_status, "device_status", torch.int32, (-1,))
     _check("mlra_cache_append", lib().mlra_cache_append(
@@ -358,7 +393,7 @@ def decode_step(cfg: Config, q_nope: torch.Tensor, q_rope: torch.Tensor, seqlens
         _need(kv_cache, "kv_cache", cfg.torch_dtype, (-1, cfg.page_size, cfg.D))
         num_pages = kv_cache.shape[0]
     else:
-        _need(kv_cache, "kv_cache", cfg.torch_dtype, (B, max_pages, cfg.D))
+        _contig_cache(kv_cache, cfg, B, max_pages)
     _check("mlra_decode_step", lib().mlra_decode_step(
         ctypes.byref(cfg), _ptr(q_nope), _ptr(q_rope), _ptr(seqlens), B, _ptr(w_uk), _ptr(w_uv),
         _ptr(kv_cache), num_pages, _ptr(page_table), int(max_pages), _ptr(out), int(on_host),
@@ -456,7 +491,7 @@ class Decoder:
 
 
 __all__ = [
-    "Config", "make_config", "lib", "absorb_q", "workspace_size", "alloc_workspace",
+    "Config", "make_config", "lib", "absorb_q", "absorb_q_rope", "workspace_size", "alloc_workspace",
     "decode_attn", "splitkv_combine", "out_proj", "combine_out_proj", "cache_append",
     "get_device_error",
     "decode_kernel_kind", "decode_attn_noalloc", "step_workspace_size", "alloc_step_workspace",

@@ -9,8 +9,9 @@ namespace mlra {
 // Dispatch entry points of the individual kernel files (host side).
 cudaError_t launch_plan(const int32_t* seqlens, int batch, int cap, int ctas_per_group, void* ws,
                         const WsLayout& L, cudaStream_t st);
+// q_abs = alpha * W_uk q_nope (alpha = 1: the plain absorption).
 cudaError_t launch_absorb(const mlra_config_t& c, const void* q_nope, const void* w_uk,
-                          float* q_abs, int batch, cudaStream_t st);
+                          float* q_abs, int batch, float alpha, cudaStream_t st);
 cudaError_t launch_combine(const mlra_config_t& c, const void* ws, const WsLayout& L, int batch,
                            float* o_latent, float* lse, cudaStream_t st);
 cudaError_t launch_out_proj(const mlra_config_t& c, const float* o_latent, const void* w_uv,
@@ -25,6 +26,12 @@ struct StageCopy {
 };
 cudaError_t launch_stage(const StageCopy* copies, int n, cudaStream_t st);
 
+// Query side of the step (k_cache.cu): q_rope_out = RoPE(alpha * q_rope) at
+// each sequence's position, in the storage dtype.
+cudaError_t launch_query_rope(const mlra_config_t& c, const void* q_rope, const int32_t* positions,
+                              float alpha, double theta, void* q_rope_out, int batch,
+                              cudaStream_t st);
+
 // Cache write (k_cache.cu).
 cudaError_t launch_cache_append(const mlra_config_t& c, const void* c_new, const void* k_rope_new,
                                 const float* gamma, float alpha_kv, float eps, double theta,
@@ -35,7 +42,7 @@ cudaError_t launch_cache_append(const mlra_config_t& c, const void* c_new, const
 // Tensor-core absorption and output projection (bf16, d_h = 128).
 bool proj_tc_supported(const mlra_config_t& c);
 cudaError_t launch_absorb_tc(const mlra_config_t& c, const void* q_nope, const void* w_uk,
-                             float* q_abs, int batch, cudaStream_t st);
+                             float* q_abs, int batch, float alpha, cudaStream_t st);
 cudaError_t launch_out_proj_tc(const mlra_config_t& c, const float* o_latent_in, const void* ws,
                                const WsLayout& L, float* o_latent_out,
                                float* lse_out, const void* w_uv, float* out, int batch,

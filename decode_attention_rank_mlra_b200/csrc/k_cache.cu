@@ -93,7 +93,62 @@ __global__ void __launch_bounds__(kCacheThreads)
   }
 }
 
+// Query side of the same step (Main Findings, variance bullet: the query is
+// scaled by alpha_q; Key Contributions #2: the decoupled RoPE query meets the
+// shared RoPE key): for every sequence s and head h,
+//   out[s, h, i], out[s, h, i + d_r/2] = the pair (i, i + d_r/2) of
+//   alpha * q_rope[s, h, :] rotated by positions[s] * theta^(-2 i / d_r),
+// the same rotation as the cache write's, so that the RoPE logit depends on the
+// distance between the query's and the key's positions only.  One CTA per
+// sequence: the d_r / 2 angles are taken once in fp64 (shared memory), then
+// every (head, pair) of the sequence is rotated in fp32 and rounded once to the
+// storage dtype.
+constexpr int kQRopeThreads = 256;
+constexpr int kMaxHalf = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kQRopeThreads)
+    query_rope_kernel(const T* __restrict__ q_rope, const int32_t* __restrict__ positions,
+                      float alpha, double theta, T* __restrict__ out, int heads, int d_r) {
+  __shared__ float cs_sm[kMaxHalf], sn_sm[kMaxHalf];
+  pdl_wait();
+  pdl_trigger();
+  const int s = blockIdx.x;
+  const int half = d_r / 2;
+  const int pos = __ldg(positions + s);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double ang = double(pos) * pow(theta, -2.0 * i / d_r);
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    cs_sm[i] = float(cs);
+    sn_sm[i] = float(sn);
+  }
+  __syncthreads();
+  const size_t base = size_t(s) * heads * d_r;
+  for (int x = threadIdx.x; x < heads * half; x += blockDim.x) {
+    const int h = x / half, i = x - h * half;
+    const T* src = q_rope + base + size_t(h) * d_r;
+    const float a = load_f(src + i) * alpha, b = load_f(src + i + half) * alpha;
+    T* dst = out + base + size_t(h) * d_r;
+    dst[i] = from_f<T>(a * cs_sm[i] - b * sn_sm[i]);
+    dst[i + half] = from_f<T>(a * sn_sm[i] + b * cs_sm[i]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_query_rope(const mlra_config_t& c, const void* q_rope, const int32_t* positions,
+                              float alpha, double theta, void* q_rope_out, int batch,
+                              cudaStream_t st) {
+  if (c.d_r % 2 != 0 || c.d_r / 2 > kMaxHalf) return cudaErrorInvalidValue;
+  if (c.dtype == MLRA_BF16)
+    return launch_pdl(query_rope_kernel<__nv_bfloat16>, dim3(batch), dim3(kQRopeThreads), 0, st,
+                      (const __nv_bfloat16*)q_rope, positions, alpha, theta,
+                      (__nv_bfloat16*)q_rope_out, c.n_heads, c.d_r);
+  return launch_pdl(query_rope_kernel<float>, dim3(batch), dim3(kQRopeThreads), 0, st,
+                    (const float*)q_rope, positions, alpha, theta, (float*)q_rope_out, c.n_heads,
+                    c.d_r);
+}
 
 cudaError_t launch_cache_append(const mlra_config_t& c, const void* c_new, const void* k_rope_new,
                                 const float* gamma, float alpha_kv, float eps, double theta,

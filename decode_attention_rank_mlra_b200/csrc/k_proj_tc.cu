@@ -50,7 +50,7 @@ template <int NT>
 __global__ void __launch_bounds__(128, 1)
     absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w,
                      const __grid_constant__ CUtensorMap map_q, float* __restrict__ q_abs,
-                     int batch, int heads, int nb, int d_cb) {
+                     int batch, int heads, int nb, int d_cb, float alpha) {
   constexpr int kA = 128 * 128;  // bytes of one 64-column box of 128 rows
   constexpr int kB = NT * 128;   // bytes of one 64-column box of NT rows
   extern __shared__ uint8_t smem_raw[];
@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(128, 1)
     for (int k = 0; k < (NT < 32 ? NT : 32); ++k) {
       const int s = s0 + c + k;
       if (s < batch)
-        q_abs[(size_t(s) * heads + h) * K + r] = good ? __uint_as_float(v[k]) : __int_as_float(0x7fc00000);
+        q_abs[(size_t(s) * heads + h) * K + r] =
+            good ? __uint_as_float(v[k]) * alpha : __int_as_float(0x7fc00000);
     }
   }
   tc_fence_before();
@@ -423,14 +424,14 @@ cudaError_t set_smem_once(Kern kern, int bytes, int* done) {
 
 template <int NT>
 cudaError_t absorb_t(const mlra_config_t& c, const CUtensorMap& mw, const CUtensorMap& mq,
-                     float* q_abs, int batch, cudaStream_t st) {
+                     float* q_abs, int batch, float alpha, cudaStream_t st) {
   static int done[64] = {0};
   const int smem = 1024 + 2 * 128 * 128 + 2 * NT * 128;
   cudaError_t e = set_smem_once(absorb_tc_kernel<NT>, smem, done);
   if (e != cudaSuccess) return e;
   dim3 grid(c.n_heads, c.n_blocks * c.d_cb / 128, (batch + NT - 1) / NT);
   return launch_pdl(absorb_tc_kernel<NT>, grid, dim3(128), smem, st, mw, mq, q_abs, batch,
-                    c.n_heads, c.n_blocks, c.d_cb);
+                    c.n_heads, c.n_blocks, c.d_cb, alpha);
 }
 
 template <bool COMBINE, int NT>
@@ -470,7 +471,7 @@ bool proj_tc_supported(const mlra_config_t& c) {
 }
 
 cudaError_t launch_absorb_tc(const mlra_config_t& c, const void* q_nope, const void* w_uk,
-                             float* q_abs, int batch, cudaStream_t st) {
+                             float* q_abs, int batch, float alpha, cudaStream_t st) {
   if (!proj_tc_supported(c) || !aligned16(q_nope) || !aligned16(w_uk)) return cudaErrorNotSupported;
   const int NT = batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 64 ? 64 : batch <= 128 ? 128 : 256;
   CUtensorMap mw, mq;
@@ -483,11 +484,11 @@ cudaError_t launch_absorb_tc(const mlra_config_t& c, const void* q_nope, const v
   if (!encode_bf16(&mw, w_uk, 2, wd, ws, wb) || !encode_bf16(&mq, q_nope, 3, qd, qs, qb))
     return cudaErrorInvalidValue;
   switch (NT) {
-    case 16: return absorb_t<16>(c, mw, mq, q_abs, batch, st);
-    case 32: return absorb_t<32>(c, mw, mq, q_abs, batch, st);
-    case 64: return absorb_t<64>(c, mw, mq, q_abs, batch, st);
-    case 128: return absorb_t<128>(c, mw, mq, q_abs, batch, st);
-    default: return absorb_t<256>(c, mw, mq, q_abs, batch, st);
+    case 16: return absorb_t<16>(c, mw, mq, q_abs, batch, alpha, st);
+    case 32: return absorb_t<32>(c, mw, mq, q_abs, batch, alpha, st);
+    case 64: return absorb_t<64>(c, mw, mq, q_abs, batch, alpha, st);
+    case 128: return absorb_t<128>(c, mw, mq, q_abs, batch, alpha, st);
+    default: return absorb_t<256>(c, mw, mq, q_abs, batch, alpha, st);
   }
 }
 

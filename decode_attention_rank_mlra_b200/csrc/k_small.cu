@@ -155,7 +155,8 @@ template <typename T>
 __global__ void __launch_bounds__(kAbsThreads) absorb_kernel(const T* __restrict__ q_nope,
                                                              const T* __restrict__ w_uk,
                                                              float* __restrict__ q_abs, int batch,
-                                                             int heads, int nb, int d_cb, int d_h) {
+                                                             int heads, int nb, int d_cb, int d_h,
+                                                             float alpha) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ float4 sq4[];  // [kSeqBlk][d_h / 4]
@@ -198,20 +199,20 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_kernel(const T* __restrict
       }
     }
   }
-  for (int s = 0; s < ns; ++s) q_abs[(size_t(s0 + s) * heads + h) * K + r] = acc[s];
+  for (int s = 0; s < ns; ++s) q_abs[(size_t(s0 + s) * heads + h) * K + r] = acc[s] * alpha;
 }
 
 cudaError_t launch_absorb(const mlra_config_t& c, const void* q_nope, const void* w_uk,
-                          float* q_abs, int batch, cudaStream_t st) {
+                          float* q_abs, int batch, float alpha, cudaStream_t st) {
   dim3 grid(c.n_heads, (c.n_blocks * c.d_cb + kAbsThreads - 1) / kAbsThreads,
             (batch + kSeqBlk - 1) / kSeqBlk);
   size_t sm = sizeof(float) * kSeqBlk * c.d_h;
   if (c.dtype == MLRA_BF16)
     return launch_pdl(absorb_kernel<__nv_bfloat16>, grid, dim3(kAbsThreads), sm, st,
                       (const __nv_bfloat16*)q_nope, (const __nv_bfloat16*)w_uk, q_abs, batch,
-                      c.n_heads, c.n_blocks, c.d_cb, c.d_h);
+                      c.n_heads, c.n_blocks, c.d_cb, c.d_h, alpha);
   return launch_pdl(absorb_kernel<float>, grid, dim3(kAbsThreads), sm, st, (const float*)q_nope,
-                    (const float*)w_uk, q_abs, batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h);
+                    (const float*)w_uk, q_abs, batch, c.n_heads, c.n_blocks, c.d_cb, c.d_h, alpha);
 }
 
 // ---------------------------------------------------------------------------

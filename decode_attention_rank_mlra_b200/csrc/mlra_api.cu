@@ -102,6 +102,16 @@ WsLayout layout_for(const mlra_config_t& c, int batch, const Grid& g) {
 
 mlra_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA; }
 
+// q_abs = alpha * W_uk q_nope on the tensor cores where they apply, else SIMT.
+mlra_status_t absorb(const mlra_config_t& c, const void* q_nope, const void* w_uk, float* q_abs,
+                     int batch, float alpha, cudaStream_t s) {
+  if (use_proj_tc(c) && aligned(q_nope, 16)) {
+    cudaError_t e = launch_absorb_tc(c, q_nope, w_uk, q_abs, batch, alpha, s);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+  }
+  return from_cuda(launch_absorb(c, q_nope, w_uk, q_abs, batch, alpha, s));
+}
+
 // Device address of the host range [p, p + bytes) when it is page-locked and
 // mapped into the current device's address space (checked at both ends), else
 // NULL, in which case no kernel ever dereferences it.
@@ -375,11 +385,34 @@ mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nope, const 
   if (!q_nope || !w_uk || !q_abs) return MLRA_ERR_INVALID_ARG;
   if (!aligned(w_uk, 16) || !aligned(q_nope, cfg->dtype == MLRA_BF16 ? 2 : 4) || !aligned(q_abs, 4))
     return MLRA_ERR_ALIGNMENT;
-  if (use_proj_tc(*cfg) && aligned(q_nope, 16)) {
-    cudaError_t e = launch_absorb_tc(*cfg, q_nope, w_uk, q_abs, batch, (cudaStream_t)stream);
-    if (e != cudaErrorNotSupported) return from_cuda(e);
-  }
-  return from_cuda(launch_absorb(*cfg, q_nope, w_uk, q_abs, batch, (cudaStream_t)stream));
+  return absorb(*cfg, q_nope, w_uk, q_abs, batch, 1.0f, (cudaStream_t)stream);
+}
+
+mlra_status_t mlra_absorb_q_rope(const mlra_config_t* cfg, const void* q_nope, const void* q_rope,
+                                 const int32_t* positions, float alpha_q, float rope_theta,
+                                 const void* w_uk, float* q_abs, void* q_rope_out, int32_t batch,
+                                 mlra_stream_t stream) {
+  mlra_status_t st = check_cfg(cfg);
+  if (st != MLRA_OK) return st;
+  if (batch < 0) return MLRA_ERR_INVALID_ARG;
+  if (batch == 0) return MLRA_OK;
+  if (!q_nope || !q_rope || !positions || !w_uk || !q_abs || !q_rope_out)
+    return MLRA_ERR_INVALID_ARG;
+  if (!(alpha_q == alpha_q) || !(rope_theta > 0.f) || cfg->d_r % 2 != 0 || cfg->d_r > 512)
+    return MLRA_ERR_INVALID_ARG;
+  const uintptr_t el = cfg->dtype == MLRA_BF16 ? 2 : 4;
+  if (!aligned(w_uk, 16) || !aligned(q_nope, el) || !aligned(q_rope, el) ||
+      !aligned(q_rope_out, el) || !aligned(q_abs, 4) || !aligned(positions, 4))
+    return MLRA_ERR_ALIGNMENT;
+  const size_t rope_bytes = size_t(batch) * cfg->n_heads * cfg->d_r * el;
+  const char* a = static_cast<const char*>(q_rope);
+  const char* b = static_cast<const char*>(q_rope_out);
+  if (a != b && a < b + rope_bytes && b < a + rope_bytes) return MLRA_ERR_INVALID_ARG;  // overlap
+  cudaStream_t s = (cudaStream_t)stream;
+  st = absorb(*cfg, q_nope, w_uk, q_abs, batch, alpha_q, s);
+  if (st != MLRA_OK) return st;
+  return from_cuda(launch_query_rope(*cfg, q_rope, positions, alpha_q, double(rope_theta),
+                                     q_rope_out, batch, s));
 }
 
 mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t batch, size_t* bytes) {

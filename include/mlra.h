@@ -107,6 +107,34 @@ MLRA_API mlra_status_t mlra_absorb_q(const mlra_config_t* cfg, const void* q_nop
                             float* q_abs, int32_t batch, mlra_stream_t stream);
 
 /*
+ * Step 1 with the query side of the calibration ("Multi-Head Low-Rank
+ * Attention", Main Findings, variance bullet: the query is scaled by
+ * alpha_q = sqrt(d / d_c'); Key Contributions #2: the decoupled RoPE query
+ * meets the one shared RoPE key):
+ *   q_abs[s, h, b, i]  = alpha_q * sum_j W_uk[b, h, i, j] * q_nope[s, h, j]   (fp32)
+ *   q_rope_out[s, h, :] = RoPE(alpha_q * q_rope[s, h, :], positions[s])       (dtype)
+ * RoPE pairs channel i with i + d_r/2 and rotates the pair by
+ * p * rope_theta^(-2i / d_r), the same rotation mlra_cache_append gives the
+ * key, so the RoPE logit depends only on the distance between the query's and
+ * the key's positions.  q_rope_out then goes to mlra_decode_attn as q_rope.
+ *   q_nope     : [batch, n_heads, d_h] dtype (before alpha_q)
+ *   q_rope     : [batch, n_heads, d_r] dtype (before alpha_q and RoPE)
+ *   positions  : [batch] int32 device memory: the query token's position
+ *                (normally seqlens[s] - 1); any int32 is a valid angle
+ *   w_uk, q_abs: as mlra_absorb_q
+ *   q_rope_out : [batch, n_heads, d_r] dtype (written); must not overlap
+ *                q_rope unless it is the same buffer (in place)
+ * The angle and its sine and cosine are taken in fp64; the rotation in fp32,
+ * rounded once to dtype.  With alpha_q = 1, q_abs equals mlra_absorb_q's bit
+ * for bit.  d_r must be even and <= 512.  batch = 0 is a no-op.
+ */
+MLRA_API mlra_status_t mlra_absorb_q_rope(const mlra_config_t* cfg, const void* q_nope,
+                                          const void* q_rope, const int32_t* positions,
+                                          float alpha_q, float rope_theta, const void* w_uk,
+                                          float* q_abs, void* q_rope_out, int32_t batch,
+                                          mlra_stream_t stream);
+
+/*
  * Workspace bytes needed by mlra_decode_attn / mlra_splitkv_combine for up to
  * `batch` sequences on the current CUDA device (depends on its SM count).
  * Writes the size to *bytes.  The workspace must be 256-byte aligned.  It holds

@@ -46,6 +46,8 @@ from .mlra_oracle import (  # noqa: F401
     SeqResult,
 )
 from .cache_oracle import (  # noqa: F401
+    q_scale,
+    query_side,
     kv_scale,
     rms_norm_blocks,
     rope,

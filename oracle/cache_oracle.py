@@ -54,6 +54,22 @@ def rope(x, pos, theta: float):
     return np.concatenate([a * cos - b * sin, a * sin + b * cos], axis=-1)
 
 
+def q_scale(d_model: int, d_cq: int) -> float:
+    """alpha_q = sqrt(d / d_c') (Main Findings, variance bullet), d_c' the
+    query latent's width."""
+    return float(np.sqrt(d_model / d_cq))
+
+
+def query_side(q_nope, q_rope, pos, alpha_q: float, theta: float):
+    """The query's share of the calibration and of RoPE (reading: alpha_q scales
+    the normalised query latent, and the query up-projection is linear, so it
+    scales both q_nope and q_rope; RoPE then rotates q_rope at the query's
+    position with the cache key's rotation).  q_nope [..., d_h], q_rope
+    [..., d_r], pos broadcast over the leading axes -> (q_nope', q_rope')."""
+    q_nope, q_rope = _f64(q_nope), _f64(q_rope)
+    return alpha_q * q_nope, rope(alpha_q * q_rope, pos, theta)
+
+
 def cache_rows(c_new, k_rope_new, gamma, n_blocks: int, alpha_kv: float, eps: float,
                pos, theta: float):
     """The new tokens' cache rows [B, n_blocks * d_cb + d_r] (fp64)."""

@@ -87,3 +87,61 @@ def test_cache_rows_layout():
     assert rows.shape == (2, 576)
     np.testing.assert_allclose(rows[0, 512:], kr[0], rtol=0, atol=0)  # position 0: unrotated
     np.testing.assert_allclose(np.sqrt(np.mean(rows[:, :128] ** 2, axis=1)), 2.0, rtol=1e-5)
+
+
+# ---- the query side: alpha_q and RoPE at the query's position ----------------
+
+def test_q_scale_matches_the_pages_formula():
+    """alpha_q = sqrt(d / d_c') (Main Findings, variance bullet)."""
+    from oracle import q_scale
+    assert q_scale(4096, 1024) == 2.0
+    assert q_scale(2048, 512) == 2.0
+    assert abs(q_scale(7168, 1536) - math.sqrt(7168 / 1536)) < 1e-15
+    assert q_scale(512, 512) == 1.0
+
+
+def test_query_side_at_position_zero_is_a_plain_scale():
+    from oracle import query_side
+    rng = np.random.default_rng(5)
+    qn, qr = rng.normal(size=(3, 4, 128)), rng.normal(size=(3, 4, 64))
+    a, b = query_side(qn, qr, np.zeros((3, 1)), 1.5, 10000.0)
+    np.testing.assert_array_equal(a, 1.5 * qn)
+    np.testing.assert_array_equal(b, 1.5 * qr)
+
+
+def test_query_alpha_scales_every_logit():
+    """Both parts of the query carry alpha_q, so the decode with the scaled query
+    equals the decode with the unscaled query and softmax scale * alpha_q."""
+    import oracle
+    from oracle import query_side
+    rng = np.random.default_rng(6)
+    h, nb, d_cb, d_h, d_r, L = 2, 4, 8, 8, 4, 9
+    qn, qr = rng.normal(size=(h, d_h)), rng.normal(size=(h, d_r))
+    c, kr = rng.normal(size=(L, nb, d_cb)), rng.normal(size=(L, d_r))
+    wk, wv = rng.normal(size=(nb, h, d_cb, d_h)), rng.normal(size=(nb, h, d_cb, d_h))
+    a = 1.7
+    qn2, qr2 = query_side(qn, qr, np.zeros(h), a, 10000.0)
+    r1 = oracle.decode_sequence(qn2, qr2, c, kr, wk, wv, 0.3, 0.5)
+    r2 = oracle.decode_sequence(qn, qr, c, kr, wk, wv, 0.3 * a, 0.5)
+    np.testing.assert_allclose(r1.out, r2.out, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(r1.lse, r2.lse, rtol=1e-13)
+
+
+def test_query_and_key_rotations_meet_at_their_distance():
+    """The RoPE logit of a query rotated at position p against a cache key
+    written at position t depends on p - t alone (the query side and the cache
+    write use the same rotation)."""
+    from oracle import query_side
+    rng = np.random.default_rng(7)
+    q, k = rng.normal(size=64), rng.normal(size=64)
+    g = np.ones(8)
+
+    def logit(p, t):
+        _, qr = query_side(np.zeros(4), q[None], np.array([p]), 1.0, 10000.0)
+        row = cache_rows(np.ones((1, 8)), k[None], g, 1, 1.0, 0.0, np.array([t]), 10000.0)
+        return float(qr[0] @ row[0, 8:])
+
+    for p, t, dp in [(10, 3, 50), (131071, 131000, -5000), (7, 7, 123)]:
+        assert abs(logit(p, t) - logit(p + dp, t + dp)) < 1e-9
+    # and it is not position-free: a different distance gives a different logit
+    assert abs(logit(10, 3) - logit(11, 3)) > 1e-6
