@@ -39,6 +39,7 @@ EXPORTS = [
     "mlra_decode_attn", "mlra_splitkv_combine", "mlra_out_proj", "mlra_get_device_error",
     "mlra_decode_kernel_kind", "mlra_decode_attn_noalloc", "mlra_combine_out_proj",
     "mlra_cache_append", "mlra_step_workspace_size", "mlra_decode_step", "mlra_absorb_q_rope",
+    "mlra_release_step_graphs",
 ]
 
 
@@ -109,6 +110,7 @@ def lib() -> ctypes.CDLL:
         "mlra_decode_attn_noalloc": (I32, [CP, P, P, P, I64, P, I32, P, I32, P, P, P, P]),
         "mlra_step_workspace_size": (I32, [CP, I32, ctypes.POINTER(SZ)]),
         "mlra_decode_step": (I32, [CP, P, P, P, I32, P, P, P, I64, P, I32, P, I32, P, SZ, P]),
+        "mlra_release_step_graphs": (I32, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -401,6 +403,12 @@ def decode_step(cfg: Config, q_nope: torch.Tensor, q_rope: torch.Tensor, seqlens
     return out
 
 
+def release_step_graphs() -> None:
+    """Destroy the CUDA graphs ``decode_step`` recorded; call only with no step
+    executing on the GPU (synchronise first)."""
+    _check("mlra_release_step_graphs", lib().mlra_release_step_graphs())
+
+
 def decode_attn_noalloc(cfg: Config, q_abs: torch.Tensor, q_rope: torch.Tensor,
                         kv_cache: torch.Tensor, page_table: Optional[torch.Tensor],
                         seqlens: torch.Tensor, max_pages: int, o_latent: torch.Tensor,
@@ -495,6 +503,6 @@ __all__ = [
     "decode_attn", "splitkv_combine", "out_proj", "combine_out_proj", "cache_append",
     "get_device_error",
     "decode_kernel_kind", "decode_attn_noalloc", "step_workspace_size", "alloc_step_workspace",
-    "decode_step",
+    "decode_step", "release_step_graphs",
     "Decoder", "MlraError", "EXPORTS", "F32", "BF16",
 ]

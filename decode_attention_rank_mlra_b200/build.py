@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmlra.so")
 SOURCES = ["mlra_api.cu", "k_small.cu", "k_decode_simt.cu", "k_decode_tc.cu", "k_decode_tc_mla.cu",
-           "k_decode_wide.cu",
+           "k_decode_mla_pair.cu", "k_decode_wide.cu",
            "k_proj_tc.cu", "k_cache.cu",
            "k_noalloc.cu"]
 HEADERS = ["mlra_internal.cuh", "dispatch.h", "tc_common.cuh", "sm100_ptx.cuh", "../../include/mlra.h"]

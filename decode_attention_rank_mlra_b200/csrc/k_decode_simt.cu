@@ -27,6 +27,18 @@ template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16
   return __bfloat162float(v);
 }
 
+// Four consecutive cache elements as fp32 (16-byte load for fp32, 8-byte for
+// bf16: every row offset and column used is a multiple of 4 elements).
+template <typename T> __device__ __forceinline__ float4 load4(const T* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) {
+  return __ldg(reinterpret_cast<const float4*>(p));
+}
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+
 template <typename T, int DCB, int DR>
 __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   constexpr int DK = DCB + DR;       // per-branch key width in the latent space
@@ -93,27 +105,31 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
     for (int t0 = tok0; t0 < tok1; t0 += kSub) {
       const int nt = min(kSub, tok1 - t0);
       __syncthreads();
-      // stage c_b | k_rope of tokens [t0, t0 + nt) (zeros past the end)
-      for (int x = tid; x < kSub * DK; x += kThreads) {
-        int tt = x / DK, k = x % DK;
-        float v = 0.f;
+      // stage c_b | k_rope of tokens [t0, t0 + nt) (zeros past the end), four
+      // elements per load, the loads of a thread independent of one another
+      constexpr int DK4 = DK / 4;
+#pragma unroll 2
+      for (int x = tid; x < kSub * DK4; x += kThreads) {
+        const int tt = x / DK4, k = (x - tt * DK4) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (tt < nt) {
-          int t = t0 + tt;
+          const int t = t0 + tt;
           long long row;
           bool ok = true;
           if (a.page_table) {
-            int pg = __ldg(a.page_table + size_t(s) * a.max_pages + t / kPageSize);
+            const int pg = __ldg(a.page_table + size_t(s) * a.max_pages + t / kPageSize);
             if (pg < 0 || pg >= a.num_pages) { ok = false; set_error(&hdr->error, MLRA_ERR_BAD_PAGE); }
             row = (long long)pg * kPageSize + (t % kPageSize);
           } else {
             row = (long long)s * a.max_pages + t;
           }
           if (ok) {
-            int col = (k < DCB) ? (b * DCB + k) : (nb * DCB + (k - DCB));
-            v = to_f32(cache[row * D + col]);
+            const int col = (k < DCB) ? (b * DCB + k) : (nb * DCB + (k - DCB));
+            v = load4<T>(cache + row * D + col);
           }
         }
-        sc[tt * RS + k] = v;
+        float* dst = sc + tt * RS + k;
+        dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
       }
       __syncthreads();
       // logits of 4 tokens per thread

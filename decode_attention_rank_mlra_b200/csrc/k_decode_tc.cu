@@ -225,11 +225,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mma_commit_warp(PVDONE(pit & 1));
     };
     while (ok && walk.next(p)) {
-      if (!wait_bar(QREADY(piece & 1), (piece >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      if (!wait_bar_warp(QREADY(piece & 1), (piece >> 1) & 1, abort_flag, err)) { ok = false; break; }
       const uint32_t qbuf = tmem + uint32_t(piece & 1) * kQBuf;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int st = it % NST, sb = it & 1;
-        if (!wait_bar(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
+        if (!wait_bar_warp(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
         const int valid = min(kTile, p.L - t * kTile);
         if (valid < kTile) {
           // zero the rows past the sequence end (whatever the cache holds there)
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           mma_commit_warp(SFULL(sb));
         }
         if (prev >= 0) {
-          if (!wait_bar(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          if (!wait_bar_warp(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           issue_pv(prev, prev_first);
         }
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // the piece's last PV goes out before the next piece's first QK: the
       // epilogue waits for it, and must not wait for the next piece's data
       if (ok && prev >= 0) {
-        if (!wait_bar(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!wait_bar_warp(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         issue_pv(prev, prev_first);
         prev = -1;
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       ++piece;
     }
     if (ok && prev >= 0) {
-      if (wait_bar(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) {
+      if (wait_bar_warp(PREADY(prev & 1), (prev >> 1) & 1, abort_flag, err)) {
         tc_fence_after();
         issue_pv(prev, prev_first);
       } else {
@@ -588,6 +588,11 @@ bool tc_supported(const mlra_config_t& c) {
 }
 
 void tc_grid(const mlra_config_t& c, int num_sms, int* n_groups, int* ctas_per_group) {
+  if (tc::mla_pair_supported(c)) {
+    *n_groups = c.n_heads / 128;
+    *ctas_per_group = tc::mla_pair_clusters(c, num_sms);
+    return;
+  }
   *n_groups = c.d_cb == 512 ? tc::mla_groups(c)
               : use_wide(c) ? tc::wide_groups(c)
                             : (c.n_blocks / g_of(c)) * (c.n_heads / hpc_of(c));
@@ -599,6 +604,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   CUtensorMap map;
   cudaError_t e = tc::make_cache_map(a, &map);
   if (e != cudaSuccess) return e;
+  if (tc::mla_pair_supported(c)) return tc::launch_decode_mla_pair(map, a, st);
   if (c.d_cb == 512) return tc::launch_decode_tc_mla(map, a, st);
   if (use_wide(c)) return tc::launch_decode_wide(map, a, st);
   switch (hpc_of(c) * 10 + g_of(c)) {

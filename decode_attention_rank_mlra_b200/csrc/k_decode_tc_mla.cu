@@ -170,10 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0, piece = 0;
     bool ok = true;
     while (ok && walk.next(p)) {
-      if (!wait_bar(QREADY, piece & 1, abort_flag, err)) { ok = false; break; }
+      if (!wait_bar_warp(QREADY, piece & 1, abort_flag, err)) { ok = false; break; }
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int st = it % kStages;
-        if (!wait_bar(FULL(st), (it / kStages) & 1, abort_flag, err)) { ok = false; break; }
+        if (!wait_bar_warp(FULL(st), (it / kStages) & 1, abort_flag, err)) { ok = false; break; }
         const int valid = min(kTile, p.L - t * kTile);
         if (valid < kTile) {
           // zero the rows past the sequence end (whatever the cache holds there)
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       0u, 0u);
         mma_commit_warp(SFULL);
         // O_q += P C_q once the probabilities are over S
-        if (!wait_bar(PREADY, it & 1, abort_flag, err)) { ok = false; break; }
+        if (!wait_bar_warp(PREADY, it & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {

@@ -14,18 +14,21 @@
 //  * warp 4 streams 64-token tiles of the cache with TMA (SWIZZLE_128B boxes of
 //    64 rows x 64 columns): the two boxes of latent block c_b and the RoPE box,
 //    into a multi-stage shared-memory ring;
-//  * warp 5 issues tcgen05.mma: S = Q . C^T with the 128 MMA rows = the 128
-//    heads, the queries in TMEM (A) and the tile K-major in shared memory (B);
-//    the fp32 absorbed query enters as bf16 hi and lo halves along K (16 MMAs
-//    over the latent block, 4 over the RoPE box, whose bf16 query is exact);
-//    then O += P . C_b with P in TMEM (A, fp16) and the tile MN-major (B);
+//  * warps 8-11 convert each arrived tile's two latent boxes from bf16 to fp16
+//    in place and zero the rows past the sequence end (exact for |c| < 65520;
+//    larger magnitudes are reported as MLRA_ERR_RANGE);
+//  * warp 13 issues tcgen05.mma: S = Q . C^T with the 128 MMA rows = the 128
+//    heads, the queries in TMEM (A) and the tile K-major in shared memory (B):
+//    8 MMAs with the fp16 query against the fp16 latent block (one row per
+//    head, scaled by a power of two that brings its largest magnitude to
+//    [2^13, 2^14)), 4 with the bf16 RoPE query (scaled by the same power of
+//    two, exactly) against the bf16 RoPE box; then O += P . C_b with P in TMEM
+//    (A, fp16) and the fp16 tile MN-major (B);
 //  * warps 0-7 (two per TMEM lane quadrant: thread = one head = one TMEM lane
 //    and one half of the tile's 64 tokens) run the online softmax of their
-//    row, write P as fp16 over S, and convert
-//    the tile's latent boxes from bf16 to fp16 in place for the product with P
-//    (an MMA's A and B share one type; fp16 P carries 11 significant bits where
-//    bf16 P carries 8, which the bf16 tolerance needs); the conversion is exact
-//    for |c| < 65520 and larger magnitudes are reported as MLRA_ERR_RANGE.
+//    row and write P as fp16 over S (an MMA's A and B share one type; fp16 P
+//    carries 11 significant bits where bf16 P carries 8, which the bf16
+//    tolerance needs).
 #include "dispatch.h"
 #include "tc_common.cuh"
 
@@ -41,30 +44,22 @@ using tc::kSmemLimit;
 using tc::wait_bar;
 using tc::wait_bar_warp;
 
-constexpr int kThreadsW = 320;                // warps 0-7 softmax, 8 TMA, 9 MMA
-constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kThreadsW = 448;                // warps 0-7 softmax, 8-11 convert, 12 TMA, 13 MMA
+constexpr int kWarpConv = 8, kWarpTma = 12, kWarpMma = 13;
 constexpr uint32_t kTmemColsW = 512;
-constexpr uint32_t kColQ = 0;                 // q hi (64 cols) | q lo (64) | q_rope (32)
-constexpr uint32_t kColQlo = 64;
-constexpr uint32_t kColQr = 128;
+constexpr uint32_t kColQ = 0;                 // fp16 query (64 cols) | bf16 RoPE query (32)
+constexpr uint32_t kColQr = 64;
 constexpr int kNS = 2;                        // S / P buffers (PV(k) follows QK(k + 1))
-constexpr uint32_t kColS = 160;               // S / P buffers: kNS x 64 columns
+constexpr uint32_t kColS = 128;               // S / P buffers: kNS x 64 columns
 constexpr uint32_t kColO = kColS + 64 * kNS;  // O accumulator: 128 columns
 constexpr int kBoxesW = 3;                    // two latent boxes + the RoPE box
 constexpr int kStageW = kBoxesW * kBoxBytes;
 constexpr int kStagesRawW = (kSmemLimit - 2048) / kStageW;
 constexpr int kStagesW = kStagesRawW > 8 ? 8 : kStagesRawW;
-constexpr int kBarsW = 2 * kStagesW + 3 * kNS + 2;
+constexpr int kBarsW = 3 * kStagesW + 3 * kNS + 2;
 constexpr int kSmemW = 1024 + kStagesW * kStageW + kBarsW * 8 + 64 + 4 * 128 * 4;
 constexpr float kPMaxW = 32768.f;             // largest P kept before a rescale (fp16)
 static_assert(kStagesW >= 3, "too few pipeline stages");
-
-// Instruction descriptor of kind::f16 with fp32 accumulation, fp16 A and B.
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major,
-                                                     bool b_mn_major) {
-  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
-         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
-}
 
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low 16 bits)
@@ -88,14 +83,15 @@ __global__ void __launch_bounds__(kThreadsW, 1)
   const uint32_t bar0 = smem_addr(bars);
   auto FULL = [&](int i) { return bar0 + 8u * i; };
   auto EMPTY = [&](int i) { return bar0 + 8u * (NST + i); };
+  auto CONV = [&](int i) { return bar0 + 8u * (2 * NST + i); };  // tile converted
   // S(k), P(k) and PV(k) use buffer k % kNS; phase parity (k / kNS) & 1.
-  auto SFULL = [&](int i) { return bar0 + 8u * (2 * NST + i); };
-  auto PREADY = [&](int i) { return bar0 + 8u * (2 * NST + kNS + i); };
+  auto SFULL = [&](int i) { return bar0 + 8u * (3 * NST + i); };
+  auto PREADY = [&](int i) { return bar0 + 8u * (3 * NST + kNS + i); };
   // PV of tile k commits to PVDONE(k % kNS): PV(k + kNS) cannot be issued
   // before this group signals P(k + kNS), so a waiter's parity is exact.
-  auto PVDONE = [&](int i) { return bar0 + 8u * (2 * NST + 2 * kNS + i); };
-  const uint32_t QREADY = bar0 + 8u * (2 * NST + 3 * kNS);  // one phase per piece
-  const uint32_t DRAIN = bar0 + 8u * (2 * NST + 3 * kNS + 1);
+  auto PVDONE = [&](int i) { return bar0 + 8u * (3 * NST + 2 * kNS + i); };
+  const uint32_t QREADY = bar0 + 8u * (3 * NST + 3 * kNS);  // one phase per piece
+  const uint32_t DRAIN = bar0 + 8u * (3 * NST + 3 * kNS + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
@@ -105,6 +101,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
     for (int i = 0; i < NST; ++i) {
       mbar_init(FULL(i), 1);
       mbar_init(EMPTY(i), 1);
+      mbar_init(CONV(i), 4);
     }
     for (int i = 0; i < kNS; ++i) {
       mbar_init(SFULL(i), 1);
@@ -186,15 +183,58 @@ __global__ void __launch_bounds__(kThreadsW, 1)
         }
       }
     }
+  } else if (warp >= kWarpConv && warp < kWarpTma) {
+    // ------------------------------------------------------------ converters
+    // The tile's two latent boxes bf16 -> fp16 in place (16-byte chunks in
+    // address order); rows past the valid tokens, latent and RoPE, become
+    // zeros, so they never depend on what the cache holds there.
+    const int ct = threadIdx.x - 32 * kWarpConv;  // 0..127
+    Piece p;
+    int it = 0;
+    bool ok = true;
+    while (ok && walk.next(p)) {
+      for (int t = p.t0; t < p.t1; ++t, ++it) {
+        const int st = it % NST;
+        if (!wait_bar_warp(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
+        const int valid = min(kTile, p.L - t * kTile);
+        uint4* base = reinterpret_cast<uint4*>(stages + st * STAGE);
+        uint32_t over = 0;
+#pragma unroll 4
+        for (int q = ct; q < 2 * 512; q += 128) {
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (((q >> 3) & 63) < valid) {
+            w = base[q];
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t h2 =
+                  pack_f16(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
+              over |= (h2 & 0x7fff7fffu) + 0x04000400u;  // inf / NaN carries into bit 15
+              wv[e] = h2;
+            }
+          }
+          base[q] = w;
+        }
+        if (valid < kTile) {
+          for (int q = ct; q < 512; q += 128)
+            if (((q >> 3) & 63) >= valid) base[2 * 512 + q] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if ((over & 0x80008000u) != 0) set_error(err, MLRA_ERR_RANGE);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(CONV(st));
+      }
+    }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop; each MMA / commit is issued by one elected
     // lane, and every wait is warp-uniform.
-    //  QK : S[heads, tokens] = Q_hi . C^T + Q_lo . C^T + Qr . Kr^T
+    //  QK : S[heads, tokens] = Q . C^T (fp16) + Qr . Kr^T (bf16)
     //       (A: queries in TMEM, B: the tile K-major)
     //  PV : O[heads, features] += P[heads, tokens] . C_b[tokens, features]
     //       (A: fp16 probabilities in TMEM over the S buffer, B: the fp16 tile MN-major)
-    constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kTile, false, false);
+    constexpr uint32_t kIdescQK = idesc_f16_f32(128, kTile, false, false);
+    constexpr uint32_t kIdescQR = idesc_bf16_f32(128, kTile, false, false);
     constexpr uint32_t kIdescPV = idesc_f16_f32(128, 128, false, true);
     const uint32_t sbase0 = smem_addr(stages);
     const uint64_t dK = smem_desc(sbase0, 16, 1024, kSwizzle128B);
@@ -223,20 +263,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
       if (!wait_bar_warp(QREADY, piece & 1, abort_flag, err)) { ok = false; break; }
       for (int t = p.t0; t < p.t1; ++t, ++it) {
         const int st = it % NST, sb = it % kNS;
-        if (!wait_bar_warp(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
-        const int valid = min(kTile, p.L - t * kTile);
-        if (valid < kTile) {
-          // zero the rows past the sequence end (whatever the cache holds there)
-          const int per_box = (kTile - valid) * 8;
-          uint8_t* sp = stages + st * STAGE;
-          for (int i = lane; i < per_box * kBoxesW; i += 32) {
-            const int bx = i / per_box, rem = i % per_box;
-            *reinterpret_cast<uint4*>(sp + bx * kBoxBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
+        if (!wait_bar_warp(CONV(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         {
           const uint64_t d = dK + uint64_t((st * STAGE) >> 4);
@@ -247,14 +274,9 @@ __global__ void __launch_bounds__(kThreadsW, 1)
                         d + uint64_t((((k >> 2) * kBoxBytes) + (k & 3) * 32) >> 4), kIdescQK,
                         k > 0 ? 1u : 0u, 0u, 0u, 0u, 0u);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ts_warp(s_acc, tmem + kColQlo + 8 * k,
-                        d + uint64_t((((k >> 2) * kBoxBytes) + (k & 3) * 32) >> 4), kIdescQK, 1u,
-                        0u, 0u, 0u, 0u);
-#pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_ts_warp(s_acc, tmem + kColQr + 8 * k,
-                        d + uint64_t((2 * kBoxBytes + k * 32) >> 4), kIdescQK, 1u, 0u, 0u, 0u, 0u);
+                        d + uint64_t((2 * kBoxBytes + k * 32) >> 4), kIdescQR, 1u, 0u, 0u, 0u, 0u);
           mma_commit_warp(SFULL(sb));
         }
         if (prev >= 0 && !issue_pv()) { ok = false; break; }
@@ -285,7 +307,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
     const int head = head0 + r;
     const int pid = 1 + q4;
     const uint32_t row_t = tmem + (uint32_t(32 * q4) << 16);
-    const float sl2 = a.cfg.softmax_scale * 1.4426950408889634f;
+    const float sl2_base = a.cfg.softmax_scale * 1.4426950408889634f;
     float* o_part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + a.L.o_part);
     float* lse_part = reinterpret_cast<float*>(static_cast<char*>(a.ws) + a.L.lse_part);
     const unsigned short* q_rope = static_cast<const unsigned short*>(a.q_rope);
@@ -294,55 +316,66 @@ __global__ void __launch_bounds__(kThreadsW, 1)
     auto pair_fail = [&](bool good) { return bar_red_or(pid, 64, !good); };
 
     // This head's queries into TMEM, half x of the latent channels and of the
-    // RoPE channels: bf16(q) | bf16(q - bf16(q)) | q_rope.
-    auto write_q = [&](const Piece& pc) {
-      const float4* q = reinterpret_cast<const float4*>(
-          a.q_abs + ((size_t(pc.s) * H + head) * nb + branch) * 128) + 16 * x;
-      float4 f[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) f[j] = __ldg(q + j);
-      uint32_t hi[32], lo[32];
+    // RoPE channels, both times 2^e (e from the largest |q_abs| of the row, so
+    // that it lands in [2^13, 2^14) as fp16): fp16(q 2^e) | q_rope 2^e (bf16,
+    // exact).  Returns 2^-e, which the softmax folds into its scale.
+    auto write_q = [&](const Piece& pc) -> float {
+      const float4* q0 = reinterpret_cast<const float4*>(
+          a.q_abs + ((size_t(pc.s) * H + head) * nb + branch) * 128);
+      float mx = 0.f;
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const float4 g = __ldg(q0 + j);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(g.x), fabsf(g.y)), fmaxf(fabsf(g.z), fabsf(g.w))));
+      }
+      int e = 0;
+      if (mx > 0.f && mx < INFINITY) {
+        const int k = int((__float_as_uint(mx) >> 23) & 0xff) - 126;  // mx in [2^(k-1), 2^k)
+        e = min(max(14 - k, -100), 100);
+      }
+      const float sc = __int_as_float((127 + e) << 23);
+      uint32_t w[32];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float v[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-          const float2 hf = __bfloat1622float2(h2);
-          hi[2 * j + e] = *reinterpret_cast<const uint32_t*>(&h2);
-          lo[2 * j + e] = tc::pack_bf16(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
-        }
+        const float4 g = __ldg(q0 + 16 * x + j);
+        w[2 * j] = pack_f16(g.x * sc, g.y * sc);
+        w[2 * j + 1] = pack_f16(g.z * sc, g.w * sc);
       }
-      tmem_st32(row_t + kColQ + 32 * x, hi);
-      tmem_st32(row_t + kColQlo + 32 * x, lo);
+      tmem_st32(row_t + kColQ + 32 * x, w);
       const uint4* qr =
           reinterpret_cast<const uint4*>(q_rope + (size_t(pc.s) * H + head) * 64) + 4 * x;
       uint32_t rr[16];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint4 u = __ldg(qr + j);
-        rr[4 * j] = u.x; rr[4 * j + 1] = u.y; rr[4 * j + 2] = u.z; rr[4 * j + 3] = u.w;
+        const uint32_t uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2)  // bf16 pair times 2^e: exact
+          rr[4 * j + e2] = tc::pack_bf16(__uint_as_float(uv[e2] << 16) * sc,
+                                         __uint_as_float(uv[e2] & 0xffff0000u) * sc);
       }
       tmem_st16(row_t + kColQr + 16 * x, rr);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(QREADY);
+      return 1.f / sc;
     };
 
     Piece p, pn;
     int it = 0;
     bool ok = walk.next(p);
-    if (ok) write_q(p);
+    float inv_sc = ok ? write_q(p) : 1.f;
     while (ok) {
+      const float sl2 = sl2_base * inv_sc;
       // m: the reference point of the exponentials, in log2 units, the same in
       // both halves of a row.  It is the first tile's max and moves only when a
       // later tile would push P past 2^15 (fp16 keeps it exactly); a stale m
       // only scales all weights alike.  l: this half's sum.
       float m = -INFINITY, l = 0.f;
       for (int t = p.t0; t < p.t1; ++t, ++it) {
-        const int sb = it % kNS, st = it % NST;
-        bool good = wait_bar(SFULL(sb), (it / kNS) & 1, abort_flag, err);
+        const int sb = it % kNS;
+        bool good = wait_bar_warp(SFULL(sb), (it / kNS) & 1, abort_flag, err);
         tc_fence_after();
         float z[32];  // raw scores of tokens 32x.. ; the scale enters with the exponent
         {
@@ -353,44 +386,6 @@ __global__ void __launch_bounds__(kThreadsW, 1)
           for (int k = 0; k < 32; ++k) z[k] = __uint_as_float(sv[k]);
         }
         const int valid = min(kTile, p.L - t * kTile);
-        // The scores are done with the tile: its latent boxes are converted to
-        // fp16 (row r: box r / 64, token row r % 64; this thread takes pieces
-        // 4x..4x+3 in swizzled order, so a quarter-warp touches different bank
-        // groups).  Rows past the valid tokens are written as zeros here too,
-        // so they never depend on which copy of the row this thread reads.
-        auto convert = [&]() {
-          uint4* row = reinterpret_cast<uint4*>(stages + st * STAGE + (r >> 6) * kBoxBytes +
-                                                (r & 63) * 128);
-          uint4 w[4];
-          if ((r & 63) >= valid) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) w[j] = make_uint4(0u, 0u, 0u, 0u);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) w[j] = row[(4 * x + j) ^ (r & 7)];
-          }
-          // an fp16 half is inf / NaN iff (h & 0x7fff) + 0x0400 carries into bit 15
-          uint32_t over = 0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w[j]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t h2 =
-                  pack_f16(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
-              over |= (h2 & 0x7fff7fffu) + 0x04000400u;
-              wv[e] = h2;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) row[(4 * x + j) ^ (r & 7)] = w[j];
-          if ((over & 0x80008000u) != 0) set_error(err, MLRA_ERR_RANGE);
-        };
-        // The two warps of a quadrant take the conversion and the exponentials
-        // in opposite orders, so one uses the conversion path while the other
-        // uses the XU pipe (the conversion has no barrier: both still meet the
-        // pair's barriers in the same order).
-        if (x == 0) convert();
         if (valid < kTile) {
 #pragma unroll
           for (int k = 0; k < 32; ++k)
@@ -431,7 +426,6 @@ __global__ void __launch_bounds__(kThreadsW, 1)
           }
         };
         exps();
-        if (x == 1) convert();
         // (ls bounds every P of this half: a P above 2^15 or a NaN fails the test)
         if (bar_red_or(pid, 64, !(ls <= kPMaxW) || !good)) {
           if (pair_fail(good)) { ok = false; break; }
@@ -448,7 +442,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
           }
           const bool any = __any_sync(0xffffffffu, alpha != 1.f);
           const int pk = it - 1;
-          const bool g2 = !any || wait_bar(PVDONE(pk % kNS), (pk / kNS) & 1, abort_flag, err);
+          const bool g2 = !any || wait_bar_warp(PVDONE(pk % kNS), (pk / kNS) & 1, abort_flag, err);
           if (pair_fail(g2)) { ok = false; break; }
           if (any) {
             tc_fence_after();
@@ -468,7 +462,6 @@ __global__ void __launch_bounds__(kThreadsW, 1)
         l += ls;
         tmem_st16(row_t + kColS + 64 * sb + 16 * x, pw);  // P over the first 32 columns of S
         tmem_wait_st();
-        fence_proxy_async_smem();  // the fp16 tile, for the PV's shared-memory reads
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(PREADY(sb));
@@ -476,11 +469,11 @@ __global__ void __launch_bounds__(kThreadsW, 1)
       if (!ok) break;
       // every QK of this piece is done: the query columns take the next piece's
       const bool has_next = walk.next(pn);
-      if (has_next) write_q(pn);
+      if (has_next) inv_sc = write_q(pn);
       // ---- epilogue: o = O / l, lse (this half: O columns 64x..64x+63)
       {
         const int pk = it - 1;
-        const bool g = wait_bar(PVDONE(pk % kNS), (pk / kNS) & 1, abort_flag, err);
+        const bool g = wait_bar_warp(PVDONE(pk % kNS), (pk / kNS) & 1, abort_flag, err);
         if (pair_fail(g)) { ok = false; break; }
       }
       tc_fence_after();

@@ -588,6 +588,19 @@ mlra_status_t mlra_decode_step(const mlra_config_t* cfg, const void* q_nope, con
   return run_step(c, (cudaStream_t)stream);
 }
 
+mlra_status_t mlra_release_step_graphs(void) {
+  std::lock_guard<std::mutex> lock(g_step_mu);
+  mlra_status_t st = MLRA_OK;
+  for (int i = 0; i < g_step_n; ++i) {
+    if (g_step_graphs[i].state == 2 && cudaGraphExecDestroy(g_step_graphs[i].exec) != cudaSuccess)
+      st = MLRA_ERR_CUDA;
+    g_step_graphs[i] = StepGraph{};
+  }
+  g_step_n = 0;
+  (void)cudaGetLastError();
+  return st;
+}
+
 mlra_status_t mlra_cache_append(const mlra_config_t* cfg, const void* c_new,
                                 const void* k_rope_new, const float* rms_gamma, float alpha_kv,
                                 float rms_eps, float rope_theta, void* kv_cache,

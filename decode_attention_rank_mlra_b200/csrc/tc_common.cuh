@@ -35,8 +35,11 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 // The same wait for a warp whose lanes go on to .sync.aligned instructions
-// (TMEM loads and stores): every lane gets the same answer, so on a timeout
-// the whole warp leaves together instead of a part of it issuing them.
+// (TMEM loads and stores): every lane tests the barrier (one instruction for
+// the warp) and gets the same answer, so on a timeout the whole warp leaves
+// together instead of a part of it issuing them.  (Measured: a single lane
+// that waits and then hands its answer to the others made the kernels
+// 15-25 % slower.)
 __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity,
                                               volatile int* abort_flag, int32_t* err) {
   const bool good = wait_bar(bar, parity, abort_flag, err);
@@ -83,6 +86,13 @@ inline bool mla_supported(const mlra_config_t& c) {
 }
 inline int mla_groups(const mlra_config_t& c) { return (c.n_heads / 64) * 2; }
 cudaError_t launch_decode_tc_mla(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st);
+
+// MLA with a multiple of 128 heads (k_decode_mla_pair.cu): clusters of two
+// CTAs, each holding half of the latent channels; ctas_per_group counts
+// clusters.
+bool mla_pair_supported(const mlra_config_t& c);
+int mla_pair_clusters(const mlra_config_t& c, int num_sms);
+cudaError_t launch_decode_mla_pair(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st);
 
 // Latent blocks of 128 channels, 128 heads x one branch per CTA
 // (k_decode_wide.cu): head counts that are multiples of 128.

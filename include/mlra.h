@@ -70,7 +70,9 @@ typedef enum {
   MLRA_ERR_TIMEOUT = 7,      /* device: a bounded wait expired                 */
   MLRA_ERR_NO_DEVICE = 8,    /* no usable sm_100 device                        */
   MLRA_ERR_RANGE = 9         /* device: a cache value of magnitude >= 65520 met
-                                the tensor-core kernel's fp16 output product   */
+                                a tensor-core kernel that takes the tile as
+                                fp16 (128 heads per CTA; MLA with a multiple
+                                of 128 heads): the result is not usable     */
 } mlra_status_t;
 
 typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype_t;
@@ -143,7 +145,10 @@ MLRA_API mlra_status_t mlra_absorb_q_rope(const mlra_config_t* cfg, const void* 
 MLRA_API mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t batch, size_t* bytes);
 
 /*
- * Step 2a: split-KV attention over the latent cache, one softmax per branch.
+ * Step 2a: split-KV attention over the latent cache, one softmax per branch
+ * ("Multi-Head Low-Rank Attention": Main Findings, the MQA-style second of the
+ * three absorbable steps; Methodology, second paragraph, attention on each
+ * latent block separately; Key Contributions #2, the shared RoPE key).
  * For every sequence s the tokens t in [0, seqlens[s]) are cut into chunks
  * (planned on the device from seqlens, balanced over the SMs); for every chunk,
  * head h and branch b it computes, over that chunk's tokens,
@@ -176,7 +181,10 @@ MLRA_API mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q
                                void* workspace, size_t workspace_bytes, mlra_stream_t stream);
 
 /*
- * Step 2b: merge the split partials of every (sequence, head, branch):
+ * Step 2b: merge the split partials of every (sequence, head, branch) -- the
+ * chunks of step 2a split one softmax over all of a sequence's tokens
+ * (Methodology, second paragraph: one softmax per branch), so their
+ * log-sum-exp merge gives that softmax's output, up to rounding:
  *   lse = log sum_k exp(lse_k);   o_lat = sum_k exp(lse_k - lse) * o_k
  *   workspace : the one passed to the preceding mlra_decode_attn (same stream)
  *   o_latent  : [batch, n_heads, n_blocks, d_cb] fp32 (written)
@@ -257,7 +265,7 @@ MLRA_API mlra_status_t mlra_step_workspace_size(const mlra_config_t* cfg, int32_
  * graph launch instead of five kernel launches; the contents of every buffer
  * may change between calls, as with direct launches).  Nothing is recorded
  * while `stream` is being captured by the caller.  The library keeps up to 64
- * such graphs per process for its lifetime.
+ * such graphs per process, until mlra_release_step_graphs.
  */
 MLRA_API mlra_status_t mlra_decode_step(const mlra_config_t* cfg, const void* q_nope,
                                         const void* q_rope, const int32_t* seqlens, int32_t batch,
@@ -266,6 +274,16 @@ MLRA_API mlra_status_t mlra_decode_step(const mlra_config_t* cfg, const void* q_
                                         int32_t max_pages, float* out, int32_t host_io,
                                         void* workspace, size_t workspace_bytes,
                                         mlra_stream_t stream);
+
+/*
+ * Destroy every CUDA graph mlra_decode_step has recorded in this process (no
+ * counterpart in the paper: the recording is a property of this library).
+ * Call it only when no mlra_decode_step call is executing on the GPU (after
+ * synchronising the streams they were made on); later calls record afresh.
+ * Returns MLRA_ERR_CUDA if a graph could not be destroyed (the record is
+ * dropped all the same).
+ */
+MLRA_API mlra_status_t mlra_release_step_graphs(void);
 
 /*
  * Cache write (the step before decode attention reads the cache; the paper

@@ -12,7 +12,7 @@ import torch
 import decode_attention_rank_mlra_b200 as mlra
 import oracle
 import workloads as W
-from parity_util import (check_close, check_lse, compare_batch, config_of, run_gpu,
+from parity_util import (check_close, check_lse, compare_batch, config_of, query_unit, run_gpu,
                          rows_logit_magnitude)
 
 pytestmark = pytest.mark.gpu
@@ -352,4 +352,5 @@ def test_full_size_sampled(name, samples):
         w_uk, _ = W.weights(spec)
         q_nope, q_rope = W.queries(spec)
         mag = rows_logit_magnitude(spec, rows, q_nope[seq], q_rope[seq], w_uk, heads)
-        check_lse(got["lse"][seq, heads].double().numpy(), ref.lse[heads], spec.dtype, mag)
+        check_lse(got["lse"][seq, heads].double().numpy(), ref.lse[heads], spec.dtype, mag,
+                  query_unit(spec))

@@ -189,3 +189,25 @@ def test_step_inside_a_caller_graph():
     torch.cuda.synchronize()
     assert torch.equal(dec.out, ref)
     assert mlra.get_device_error(dec.workspace) == 0
+
+
+def test_released_graphs_record_again():
+    """The same call (same pointers) runs directly, is recorded, is replayed;
+    after mlra_release_step_graphs it records afresh: the same result bit for
+    bit every time."""
+    inp = _inputs("mlra4_bf16_b64_h32_l16384_paged", [300, 70])
+    cfg = config_of(inp.spec)
+    dec = mlra.Decoder(cfg, inp.spec.batch, inp.device)
+    out = torch.empty(dec.out.shape, dtype=torch.float32, device=inp.device)
+    outs = []
+    for k in range(6):
+        if k == 3:
+            torch.cuda.synchronize()
+            mlra.release_step_graphs()
+        out.fill_(float("nan"))
+        dec.step(inp.q_nope, inp.q_rope, inp.seqlens, inp.w_uk, inp.w_uv, inp.kv_cache,
+                 inp.page_table, _max_pages(inp), out=out)
+        assert mlra.get_device_error(dec.workspace) == 0
+        outs.append(out.cpu().clone())
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])

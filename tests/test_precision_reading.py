@@ -35,6 +35,13 @@ def _round(x, mode):
         return _bf16(x)
     if mode == "fp16":
         return np.asarray(x, np.float32).astype(np.float16).astype(np.float64)
+    if mode == "fp16s":
+        # fp16 after a power-of-two scale per row (last axis) that brings the
+        # row's largest magnitude to [2^13, 2^14), then scaled back (exact)
+        mx = np.max(np.abs(x), axis=-1, keepdims=True)
+        e = np.where(mx > 0, 14 - (np.floor(np.log2(np.where(mx > 0, mx, 1.0))) + 1), 0)
+        sc = np.exp2(e)
+        return (np.asarray(x * sc, np.float32).astype(np.float16).astype(np.float64)) / sc
     raise ValueError(mode)
 
 
@@ -76,6 +83,17 @@ def test_kernel_roundings_are_inside_the_bound(name):
     for pmode in ("hilo", "fp16"):
         mx, mn = _errors(name, "hilo", pmode)
         assert mx <= BF16_MAX / 3 and mn <= BF16_MEAN / 2, (pmode, mx, mn)
+
+
+@pytest.mark.parametrize("name", ["mlra4_bf16_b8_h128_l131072_paged",
+                                  "mla_bf16_b8_h128_l131072_paged"])
+def test_fp16_queries_of_the_128_head_kernels_are_inside_the_bound(name):
+    """The 128-head MLRA-4 and MLA kernels take the query as one fp16 row per
+    head (scaled by a power of two per row: per branch for MLRA-4, the whole
+    512-channel row for MLA) against an fp16 copy of the tile, with fp16
+    probabilities: inside the bound with the margin the tests need."""
+    mx, mn = _errors(name, "fp16s", "fp16")
+    assert mx <= BF16_MAX / 3 and mn <= 0.6 * BF16_MEAN, (mx, mn)
 
 
 @pytest.mark.parametrize("name", ["mlra4_bf16_b8_h128_l131072_paged",
