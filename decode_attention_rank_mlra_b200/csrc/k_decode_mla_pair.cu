@@ -30,13 +30,13 @@
 // Precision: queries as fp16 (one row per head, scaled per head by a power of
 // two that brings the row's largest magnitude to [2^13, 2^14)), the latent
 // tile converted bf16 -> fp16 in place by four converter warps before the
-// scores (exact for |c| < 65520; larger magnitudes are reported as
+// scores (exact for 2^-17 <= |c| < 65520; larger magnitudes are reported as
 // MLRA_ERR_RANGE), fp16 probabilities, fp32 accumulation; the RoPE part stays
 // bf16 x bf16 (the query scaled by the same power of two, exactly).
 //
 // Warps: 0-7 softmax (warp w: TMEM quadrant w & 3, token half w >> 2; "own"
-// when the quadrant holds this CTA's heads, "relay" otherwise), 8-11 convert,
-// 12 TMA, 13 MMA.
+// when the quadrant holds this CTA's heads, "relay" otherwise), 8 and 10-12 convert,
+// 9 MMA, 13 TMA.
 #include "tc_common.cuh"
 
 #include <cuda_fp16.h>
@@ -49,7 +49,12 @@ namespace {
 using namespace ptx;
 
 constexpr int kThreads = 448;
-constexpr int kWarpConv = 8, kWarpTma = 12, kWarpMma = 13;
+// The MMA-issuing warp stalls its scheduler while the tensor pipe accepts its
+// instructions, so no converter shares that scheduler (warp w runs on
+// scheduler w % 4): MMA warp 9, TMA warp 13, converters 8, 10, 11, 12.
+constexpr int kWarpTma = 13, kWarpMma = 9;
+__device__ __forceinline__ bool is_conv(int w) { return w == 8 || (w >= 10 && w <= 12); }
+__device__ __forceinline__ int conv_index(int w) { return w == 8 ? 0 : w - 9; }
 constexpr int kBoxes = 5;                       // 4 latent boxes of this CTA's half + RoPE
 constexpr int kStage = kBoxes * kBoxBytes;      // 40 KB
 constexpr int kStages = 3;
@@ -247,12 +252,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp >= kWarpConv && warp < kWarpTma) {
+  } else if (is_conv(warp)) {
     // ------------------------------------------------------------ converters
     // Each tile's four latent boxes bf16 -> fp16 in place (16-byte chunks, any
     // order); rows past the valid tokens (latent and RoPE) become zeros, so
     // they never depend on what the cache holds there.
-    const int ct = threadIdx.x - 32 * kWarpConv;  // 0..127
+    const int ct = 32 * conv_index(warp) + lane;  // 0..127
     Piece p;
     int it = 0;
     bool ok = true;
@@ -264,29 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const int valid = min(kTile, p.L - t * kTile);
-        uint4* base = reinterpret_cast<uint4*>(stages + st * kStage);
-        uint32_t over = 0;
-#pragma unroll 4
-        for (int q = ct; q < 4 * 512; q += 128) {
-          const int row = (q >> 3) & 63;
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (row < valid) {
-            w = base[q];
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t h2 =
-                  pack_h2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
-              over |= (h2 & 0x7fff7fffu) + 0x04000400u;  // inf / NaN carries into bit 15
-              wv[e] = h2;
-            }
-          }
-          base[q] = w;
-        }
-        if (valid < kTile) {
-          for (int q = ct; q < 512; q += 128)
-            if (((q >> 3) & 63) >= valid) base[4 * 512 + q] = make_uint4(0u, 0u, 0u, 0u);
-        }
+        const uint32_t base = smem_addr(stages + st * kStage);
+        const uint32_t over = convert_stage<4 * 512, 128>(base, ct, valid);
+        if (valid < kTile) zero_box_rows<128>(base + 4 * kBoxBytes, ct, valid);
         if ((over & 0x80008000u) != 0) set_error(err, MLRA_ERR_RANGE);
         fence_proxy_async_smem();
         __syncwarp();

@@ -11,13 +11,13 @@
 // absorbed "MQA-style" step of Main Findings ("three absorbable steps").
 //
 // How (one CTA per SM, persistent over a share of the tile stream):
-//  * warp 4 streams 64-token tiles of the cache with TMA (SWIZZLE_128B boxes of
+//  * warp 12 streams 64-token tiles of the cache with TMA (SWIZZLE_128B boxes of
 //    64 rows x 64 columns): the two boxes of latent block c_b and the RoPE box,
 //    into a multi-stage shared-memory ring;
-//  * warps 8-11 convert each arrived tile's two latent boxes from bf16 to fp16
-//    in place and zero the rows past the sequence end (exact for |c| < 65520;
-//    larger magnitudes are reported as MLRA_ERR_RANGE);
-//  * warp 13 issues tcgen05.mma: S = Q . C^T with the 128 MMA rows = the 128
+//  * warps 8, 10, 11, 13 convert each arrived tile's two latent boxes from bf16 to fp16
+//    in place and zero the rows past the sequence end (exact for
+//    2^-17 <= |c| < 65520; larger magnitudes are reported as MLRA_ERR_RANGE);
+//  * warp 9 issues tcgen05.mma: S = Q . C^T with the 128 MMA rows = the 128
 //    heads, the queries in TMEM (A) and the tile K-major in shared memory (B):
 //    8 MMAs with the fp16 query against the fp16 latent block (one row per
 //    head, scaled by a power of two that brings its largest magnitude to
@@ -44,12 +44,18 @@ using tc::kSmemLimit;
 using tc::wait_bar;
 using tc::wait_bar_warp;
 
-constexpr int kThreadsW = 448;                // warps 0-7 softmax, 8-11 convert, 12 TMA, 13 MMA
-constexpr int kWarpConv = 8, kWarpTma = 12, kWarpMma = 13;
+constexpr int kThreadsW = 448;                // warps 0-7 softmax, 8, 10, 11, 13 convert, 9 MMA, 12 TMA
+// One converter warp per scheduler (warp w runs on scheduler w % 4), beside
+// the two softmax warps there: converters 8, 10, 11, 13, MMA warp 9, TMA warp 12.
+constexpr int kWarpTma = 12, kWarpMma = 9;
+__device__ __forceinline__ bool is_conv(int w) { return w == 8 || w == 10 || w == 11 || w == 13; }
+__device__ __forceinline__ int conv_index(int w) { return w == 8 ? 0 : w == 13 ? 3 : w - 9; }
 constexpr uint32_t kTmemColsW = 512;
 constexpr uint32_t kColQ = 0;                 // fp16 query (64 cols) | bf16 RoPE query (32)
 constexpr uint32_t kColQr = 64;
-constexpr int kNS = 2;                        // S / P buffers (PV(k) follows QK(k + 1))
+constexpr int kNS = 4;                        // S / P buffers (PV(k) follows QK(k + kLook))
+constexpr int kLook = 2;                      // QKs issued ahead of the oldest pending PV
+static_assert(kLook < kNS, "QK(k + kNS) reuses the buffer that PV(k) reads");
 constexpr uint32_t kColS = 128;               // S / P buffers: kNS x 64 columns
 constexpr uint32_t kColO = kColS + 64 * kNS;  // O accumulator: 128 columns
 constexpr int kBoxesW = 3;                    // two latent boxes + the RoPE box
@@ -183,12 +189,12 @@ __global__ void __launch_bounds__(kThreadsW, 1)
         }
       }
     }
-  } else if (warp >= kWarpConv && warp < kWarpTma) {
+  } else if (is_conv(warp)) {
     // ------------------------------------------------------------ converters
     // The tile's two latent boxes bf16 -> fp16 in place (16-byte chunks in
     // address order); rows past the valid tokens, latent and RoPE, become
     // zeros, so they never depend on what the cache holds there.
-    const int ct = threadIdx.x - 32 * kWarpConv;  // 0..127
+    const int ct = 32 * conv_index(warp) + lane;  // 0..127
     Piece p;
     int it = 0;
     bool ok = true;
@@ -197,28 +203,9 @@ __global__ void __launch_bounds__(kThreadsW, 1)
         const int st = it % NST;
         if (!wait_bar_warp(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
         const int valid = min(kTile, p.L - t * kTile);
-        uint4* base = reinterpret_cast<uint4*>(stages + st * STAGE);
-        uint32_t over = 0;
-#pragma unroll 4
-        for (int q = ct; q < 2 * 512; q += 128) {
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (((q >> 3) & 63) < valid) {
-            w = base[q];
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t h2 =
-                  pack_f16(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
-              over |= (h2 & 0x7fff7fffu) + 0x04000400u;  // inf / NaN carries into bit 15
-              wv[e] = h2;
-            }
-          }
-          base[q] = w;
-        }
-        if (valid < kTile) {
-          for (int q = ct; q < 512; q += 128)
-            if (((q >> 3) & 63) >= valid) base[2 * 512 + q] = make_uint4(0u, 0u, 0u, 0u);
-        }
+        const uint32_t base = smem_addr(stages + st * STAGE);
+        const uint32_t over = tc::convert_stage<2 * 512, 128>(base, ct, valid);
+        if (valid < kTile) tc::zero_box_rows<128>(base + 2 * kBoxBytes, ct, valid);
         if ((over & 0x80008000u) != 0) set_error(err, MLRA_ERR_RANGE);
         fence_proxy_async_smem();
         __syncwarp();
@@ -241,22 +228,29 @@ __global__ void __launch_bounds__(kThreadsW, 1)
     const uint64_t dMN = smem_desc(sbase0, kBoxBytes, 1024, kSwizzle128B);
     Piece p;
     int it = 0, piece = 0;
-    int prev = -1;            // tile whose PV is still to be issued
-    bool prev_first = false;  // ...and whether it opens its piece
+    // tiles whose PV is still to be issued: npend consecutive tiles from
+    // `oldest`; bit j of first_mask: pending tile j opens its piece (its PV
+    // then overwrites O)
+    int oldest = 0, npend = 0;
+    uint32_t first_mask = 0;
     bool ok = true;
-    // PV(prev): after QK(prev + 1), so the softmax of tile prev overlaps it
+    // PV of the oldest pending tile: issued after QK of the kLook tiles that
+    // follow it, so those scores are ready while its softmax runs
     auto issue_pv = [&]() -> bool {
-      if (!wait_bar_warp(PREADY(prev % kNS), (prev / kNS) & 1, abort_flag, err)) return false;
+      const int k0 = oldest;
+      if (!wait_bar_warp(PREADY(k0 % kNS), (k0 / kNS) & 1, abort_flag, err)) return false;
       tc_fence_after();
-      const uint64_t d = dMN + uint64_t(((prev % NST) * STAGE) >> 4);
-      const uint32_t a_p = tmem + kColS + 64 * (prev % kNS);
+      const uint64_t d = dMN + uint64_t(((k0 % NST) * STAGE) >> 4);
+      const uint32_t a_p = tmem + kColS + 64 * (k0 % kNS);
 #pragma unroll
       for (int k = 0; k < kTile / 16; ++k)
         mma_ts_warp(tmem + kColO, a_p + 8 * k, d + uint64_t((k * 16 * 128) >> 4), kIdescPV,
-                    (prev_first && k == 0) ? 0u : 1u, 0u, 0u, 0u, 0u);
-      mma_commit_warp(EMPTY(prev % NST));
-      mma_commit_warp(PVDONE(prev % kNS));
-      prev = -1;
+                    ((first_mask & 1u) && k == 0) ? 0u : 1u, 0u, 0u, 0u, 0u);
+      mma_commit_warp(EMPTY(k0 % NST));
+      mma_commit_warp(PVDONE(k0 % kNS));
+      ++oldest;
+      first_mask >>= 1;
+      --npend;
       return true;
     };
     while (ok && walk.next(p)) {
@@ -279,13 +273,15 @@ __global__ void __launch_bounds__(kThreadsW, 1)
                         d + uint64_t((2 * kBoxBytes + k * 32) >> 4), kIdescQR, 1u, 0u, 0u, 0u, 0u);
           mma_commit_warp(SFULL(sb));
         }
-        if (prev >= 0 && !issue_pv()) { ok = false; break; }
-        prev = it;
-        prev_first = (t == p.t0);
+        if (npend == 0) oldest = it;
+        first_mask |= uint32_t(t == p.t0) << npend;
+        ++npend;
+        if (npend > kLook && !issue_pv()) { ok = false; break; }
       }
-      // the piece's last PV goes out before the next piece's first QK: the
-      // epilogue waits for it, and the next piece's queries wait for the epilogue
-      if (ok && prev >= 0 && !issue_pv()) ok = false;
+      // the piece's last PVs go out before the next piece's first QK: the
+      // epilogue waits for them, and the next piece's queries wait for the epilogue
+      while (ok && npend > 0)
+        if (!issue_pv()) ok = false;
       ++piece;
     }
     if (!ok) {

@@ -7,6 +7,7 @@
 #include "sm100_ptx.cuh"
 
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 
 namespace mlra {
 namespace tc {
@@ -49,6 +50,65 @@ __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity,
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Eight bf16 values (one 16-byte chunk) -> fp16 in place, round to nearest:
+// exact for 2^-17 <= |c| < 65520 (bf16's 8 significant bits fit fp16's), a
+// smaller magnitude lands on fp16's subnormal grid of 2^-24.  Returns bits 15 /
+// 31 set when a value became inf or NaN, i.e. left the fp16 range.
+__device__ __forceinline__ uint32_t bf16x8_to_f16(uint4& w) {
+  uint32_t over = 0;
+  uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __half2 h = __floats2half2_rn(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
+    const uint32_t h2 = *reinterpret_cast<uint32_t*>(&h);
+    over |= (h2 & 0x7fff7fffu) + 0x04000400u;  // inf / NaN carries into bit 15
+    wv[e] = h2;
+  }
+  return over;
+}
+
+// Converter step over one stage: the chunks q = ct, ct + kConvThreads, ... <
+// n_chunks of the latent boxes at shared address `base` (64 rows of 128 bytes
+// per box, chunk q in row (q / 8) mod 64), bf16 -> fp16 in place; rows at or
+// past `valid` become zeros.  Two chunks in flight per thread.
+template <int kChunks, int kConvThreads>
+__device__ __forceinline__ uint32_t convert_stage(uint32_t base, int ct, int valid) {
+  static_assert(kChunks % (2 * kConvThreads) == 0, "chunks split evenly in pairs");
+  uint32_t over = 0;
+  if (valid >= 64) {
+#pragma unroll
+    for (int i = 0; i < kChunks / kConvThreads; i += 2) {
+      const uint32_t a0 = base + 16u * uint32_t(ct + kConvThreads * i);
+      const uint32_t a1 = a0 + 16u * kConvThreads;
+      uint4 w0 = ptx::lds128(a0), w1 = ptx::lds128(a1);
+      over |= bf16x8_to_f16(w0);
+      over |= bf16x8_to_f16(w1);
+      ptx::sts128(a0, w0);
+      ptx::sts128(a1, w1);
+    }
+  } else {
+#pragma unroll 1
+    for (int q = ct; q < kChunks; q += kConvThreads) {
+      const uint32_t a0 = base + 16u * uint32_t(q);
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (((q >> 3) & 63) < valid) {
+        w = ptx::lds128(a0);
+        over |= bf16x8_to_f16(w);
+      }
+      ptx::sts128(a0, w);
+    }
+  }
+  return over;
+}
+
+// Zero the rows at or past `valid` of the 64 x 128-byte box at `base`.
+template <int kConvThreads>
+__device__ __forceinline__ void zero_box_rows(uint32_t base, int ct, int valid) {
+#pragma unroll 1
+  for (int q = ct; q < 512; q += kConvThreads)
+    if (((q >> 3) & 63) >= valid) ptx::sts128(base + 16u * uint32_t(q), make_uint4(0u, 0u, 0u, 0u));
 }
 
 // The cache as a 2-D bf16 tensor [rows, D] (rows = pages * 64, or batch *
