@@ -35,8 +35,8 @@
 // bf16 x bf16 (the query scaled by the same power of two, exactly).
 //
 // Warps: 0-7 softmax (warp w: TMEM quadrant w & 3, token half w >> 2; "own"
-// when the quadrant holds this CTA's heads, "relay" otherwise), 8 and 10-12 convert,
-// 9 MMA, 13 TMA.
+// in quadrants 2, 3, which hold this CTA's heads, "relay" in quadrants 0, 1),
+// 8, 9, 12, 13 convert, 10 TMA, 11 MMA.
 #include "tc_common.cuh"
 
 #include <cuda_fp16.h>
@@ -49,12 +49,13 @@ namespace {
 using namespace ptx;
 
 constexpr int kThreads = 448;
-// The MMA-issuing warp stalls its scheduler while the tensor pipe accepts its
-// instructions, so no converter shares that scheduler (warp w runs on
-// scheduler w % 4): MMA warp 9, TMA warp 13, converters 8, 10, 11, 12.
-constexpr int kWarpTma = 13, kWarpMma = 9;
-__device__ __forceinline__ bool is_conv(int w) { return w == 8 || (w >= 10 && w <= 12); }
-__device__ __forceinline__ int conv_index(int w) { return w == 8 ? 0 : w - 9; }
+// Warp w runs on scheduler w % 4.  Each CTA keeps its own heads' rows in TMEM
+// lanes 64-127 (quadrants 2, 3), so its softmax exponentials run on schedulers
+// 2 and 3; the converters (whose bf16 -> fp16 conversions share the
+// exponentials' unit) sit on schedulers 0 and 1 with the relay warps.
+constexpr int kWarpTma = 10, kWarpMma = 11;
+__device__ __forceinline__ bool is_conv(int w) { return w == 8 || w == 9 || w == 12 || w == 13; }
+__device__ __forceinline__ int conv_index(int w) { return (w & 1) + 2 * ((w >> 2) & 1); }
 constexpr int kBoxes = 5;                       // 4 latent boxes of this CTA's half + RoPE
 constexpr int kStage = kBoxes * kBoxBytes;      // 40 KB
 constexpr int kStages = 3;
@@ -355,10 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax warps 0-7
     const int qd = warp & 3, x = warp >> 2;
-    const bool own = (qd >> 1) == rank;
-    const int r = 32 * qd + lane;         // TMEM lane = row = head within the group
+    // TMEM lane r holds head (r + 64 (1 - rank)) mod 128 of the group: this
+    // CTA's own heads in lanes 64-127, the partner's in lanes 0-63
+    const bool own = (qd >> 1) == 1;
+    const int r = 32 * qd + lane;         // TMEM lane = MMA row
     const int rl = r & 63;                // row within the 64 heads of one CTA
-    const int head = head0 + r;
+    const int head = head0 + ((r + 64 * (1 - rank)) & 127);
     const int pid = 1 + qd;               // named barrier of the quadrant's two warps
     const uint32_t row_t = tmem + (uint32_t(32 * qd) << 16);
     const float sl2_base = a.cfg.softmax_scale * 1.4426950408889634f;
@@ -487,10 +490,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                           64 * (qd & 1);
       const float alpha = side[lane];
       if (last) inv_l = side[32 + lane];
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(peer_pmsge0 + 8u * sb);  // buffer read
       tmem_st16(row_t + kColS + 64 * sb + 16 * x, pw);
-      if (__any_sync(0xffffffffu, alpha != 1.f) && may_rescale) {
+      // (the store above and the vote below consume every value read from the
+      // message: the buffer may go back to the partner; inv_l is never negative)
+      const bool resc = __any_sync(0xffffffffu, alpha != 1.f || inv_l < 0.f);
+      if (lane == 0) mbar_arrive_remote(peer_pmsge0 + 8u * sb);  // buffer read
+      if (resc && may_rescale) {
         const int pk = itx - 1;
         if (!wait_bar_warp(BAR(kBPvDone + (pk & 1)), (pk >> 1) & 1, abort_flag, err)) return false;
         tc_fence_after();
@@ -547,8 +552,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 32; ++k) z[k] += __uint_as_float(sv[k]);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(peer_smsge0 + 8u * sb);  // message read
           if (valid < kTile) {
 #pragma unroll
             for (int k = 0; k < 32; ++k)
@@ -584,7 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           };
           exps();
           float alpha = 1.f;
-          if (bar_red_or(pid, 64, !(ls <= kPMax))) {
+          const bool over = bar_red_or(pid, 64, !(ls <= kPMax));
+          // (ls, an input of the vote, depends on every value read from the
+          // message: the buffer may go back to the partner)
+          if (lane == 0) mbar_arrive_remote(peer_smsge0 + 8u * sb);  // message read
+          if (over) {
             // rare: a score far above m (or a NaN): raise m to this tile's row
             // max, rescale l and this CTA's O rows of these heads (the partner
             // rescales its own from alpha), redo the tile
