@@ -8,7 +8,7 @@ already resident in HBM.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference] [--no-cpu-baseline]
-                  [--per-config all|none|NAME,NAME...]
+                  [--per-config all|none|NAME,NAME...] [--batch N]
 
 Prints ONE JSON line (rank 0).  The headline is the largest single-GPU
 workload (the ragged batch of 128 sequences, 4.9 GB of cache): value = decode
@@ -65,7 +65,18 @@ def parse(argv=None):
                    help="workloads measured besides the headline: all, none, or a comma list")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="bound on the oracle's CPU work for the baseline sample")
+    p.add_argument("--batch", type=int, default=0,
+                   help="run the workload with this many sequences instead (same lengths, "
+                        "same layout): a smaller case of the same kernels, for profiling")
     return p.parse_args(argv)
+
+
+def workload_spec(W, args):
+    """The named workload, or (--batch) a smaller case of it with that many sequences."""
+    spec = W.WORKLOADS[args.workload]
+    if args.batch > 0 and args.batch != spec.batch:
+        spec = W.scaled_down(spec, args.batch, seqlen=spec.seqlen, ragged=spec.ragged)
+    return spec
 
 
 def dist_env():
@@ -598,7 +609,7 @@ def run_ours(args):
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", torch.cuda.current_device())
-    spec = W.WORKLOADS[args.workload]
+    spec = workload_spec(W, args)
     stream = torch.cuda.current_stream()
     sampler = ClockSampler(dev.index if world == 1 else local)
     sampler.start()
@@ -671,7 +682,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return None
-    spec = W.WORKLOADS[args.workload]
+    spec = workload_spec(W, args)
     per_step = min(3.0, max(0.02, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(spec, per_step)

@@ -623,7 +623,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               lse_part[size_t(p.slot) * H + head] =
                   l_tot > 0.f ? (m + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
           }
-          tmem_st16(row_t + kColS + 64 * sb + 16 * x, pw);  // P over S
           {  // the partner's relay has read P(it - 2): both copies of buffer sb are free
             const bool g3 = wait_cl_warp(BAR(kBPMsgE + sb), ((it >> 1) & 1) ^ 1, abort_flag, err);
             if (pair_fail(g3)) { ok = false; break; }
@@ -653,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     uint32_t(qd & 1) * 256u,
                                 so, 256u, fb);
           }
+          tmem_st16(row_t + kColS + 64 * sb + 16 * x, pw);  // P over S
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
