@@ -42,6 +42,8 @@ using tc::wait_bar;
 using tc::wait_bar_warp;
 
 constexpr int kThreadsTC = 192;              // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr int kPrefetchAhead = 6;            // tiles before a piece's end
+constexpr int kPrefetchTiles = 4;            // first tiles of the next sequence
 constexpr uint32_t kTmemCols = 512;
 // Queries are double-buffered by piece: buffer b at b * kQBuf holds the q_abs
 // rows (bf16 pairs, 64 columns) and then the q_rope rows (32 columns).
@@ -143,12 +145,38 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if (lane == 0) {
       prefetch_tensormap(&tmap);
       const uint64_t evict_first = policy_evict_first();  // the cache is streamed once
+      // The first tiles of a new sequence arrive slowly (cold pages): a few
+      // tiles before a piece that another piece follows ends, the first tiles
+      // of the next sequence are prefetched into L2.
+      const size_t row_bytes = size_t(a.cfg.n_blocks * a.cfg.d_cb + a.cfg.d_r) * 2;
+      auto prefetch_head = [&](int s2) {
+        if (s2 >= a.batch) return;
+        const int L2 = min(max(__ldg(a.seqlens + s2), 0), a.cap);
+        const int nt = min((L2 + kTile - 1) / kTile, kPrefetchTiles);
+        for (int j = 0; j < nt; ++j) {
+          int64_t row;
+          int rows = kTile;
+          if (a.page_table) {
+            const int pg = __ldg(a.page_table + size_t(s2) * a.max_pages + j);
+            if (pg < 0 || pg >= a.num_pages) continue;
+            row = int64_t(pg) * kPageSize;
+          } else {
+            row = int64_t(s2) * a.max_pages + int64_t(j) * kTile;
+            rows = min(kTile, a.max_pages - j * kTile);  // the allocation ends with the last row
+          }
+          bulk_prefetch_l2(static_cast<const char*>(a.kv_cache) + row * row_bytes,
+                           uint32_t(rows * row_bytes));
+        }
+      };
       Piece p;
       int it = 0;
       bool ok = true;
       while (ok && walk.next(p)) {
+        const bool more = walk.gt < walk.end;  // another piece follows in this share
+        const int t_pf = max(p.t0, p.t1 - kPrefetchAhead);
         for (int t = p.t0; t < p.t1; ++t, ++it) {
           const int st = it % NST;
+          if (more && t == t_pf) prefetch_head(p.s + 1);
           if (!wait_bar(EMPTY(st), ((it / NST) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
           int row;
           if (a.page_table) {

@@ -84,6 +84,11 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 __device__ __forceinline__ void prefetch_l2_evict_last(const void* ptr) {
   asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(ptr) : "memory");
 }
+// Bulk prefetch of [ptr, ptr + bytes) into L2 (16-byte aligned address, size a
+// multiple of 16); nothing is written anywhere.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
