@@ -31,7 +31,8 @@
 // two that brings the row's largest magnitude to [2^13, 2^14)), the latent
 // tile converted bf16 -> fp16 in place by four converter warps before the
 // scores (exact for 2^-17 <= |c| < 65520; larger magnitudes are reported as
-// MLRA_ERR_RANGE), fp16 probabilities, fp32 accumulation; the RoPE part stays
+// MLRA_ERR_RANGE, and the 64-head MLA kernel launched after this one then
+// recomputes the call), fp16 probabilities, fp32 accumulation; the RoPE part stays
 // bf16 x bf16 (the query scaled by the same power of two, exactly).
 //
 // Warps: 0-7 softmax (warp w: TMEM quadrant w & 3, token half w >> 2; "own"

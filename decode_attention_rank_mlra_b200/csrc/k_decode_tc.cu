@@ -94,7 +94,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
-  int32_t* err = &hdr->error;
+  if (a.range_fallback) {
+    // after the 128-head kernel's grid: every thread reads its final error word
+    pdl_wait();
+    if (*reinterpret_cast<volatile int32_t*>(&hdr->error) != MLRA_ERR_RANGE) return;
+  }
+  int32_t* err = a.range_fallback ? &hdr->fallback_error : &hdr->error;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
@@ -554,6 +559,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if (a.range_fallback && threadIdx.x == 0) {
+    // the last CTA out replaces MLRA_ERR_RANGE by this launch's own outcome
+    __threadfence();
+    if (atomicAdd(&hdr->fallback_done, 1) == int(gridDim.x) - 1)
+      atomicCAS(&hdr->error, MLRA_ERR_RANGE,
+                *reinterpret_cast<volatile int32_t*>(&hdr->fallback_error));
+  }
 }
 
 // Heads per CTA (a head group) and branches per CTA: the 128 MMA rows hold
@@ -627,14 +639,8 @@ void tc_grid(const mlra_config_t& c, int num_sms, int* n_groups, int* ctas_per_g
   *ctas_per_group = num_sms / *n_groups > 0 ? num_sms / *n_groups : 1;
 }
 
-cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_rows(const CUtensorMap& map, const DecodeArgs& a, cudaStream_t st) {
   const mlra_config_t& c = a.cfg;
-  CUtensorMap map;
-  cudaError_t e = tc::make_cache_map(a, &map);
-  if (e != cudaSuccess) return e;
-  if (tc::mla_pair_supported(c)) return tc::launch_decode_mla_pair(map, a, st);
-  if (c.d_cb == 512) return tc::launch_decode_tc_mla(map, a, st);
-  if (use_wide(c)) return tc::launch_decode_wide(map, a, st);
   switch (hpc_of(c) * 10 + g_of(c)) {
     case 164: return launch_t<4, 16>(map, a, st);
     case 162: return launch_t<2, 16>(map, a, st);
@@ -644,6 +650,35 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
     case 641: return launch_t<1, 64>(map, a, st);
   }
   return cudaErrorInvalidValue;
+}
+
+// The 128-head kernels carry the tile as fp16 and report a cache value of
+// magnitude >= 65520 (MLRA_ERR_RANGE).  Each is followed by a launch of a
+// kernel that keeps the tile in bf16 (head-rows for MLRA with 128 heads, the
+// 64-head MLA kernel for MLA) on the same plan and slots: its CTAs return at
+// once unless the word holds MLRA_ERR_RANGE, and otherwise recompute the call.
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
+  const mlra_config_t& c = a.cfg;
+  CUtensorMap map;
+  cudaError_t e = tc::make_cache_map(a, &map);
+  if (e != cudaSuccess) return e;
+  DecodeArgs f = a;
+  f.range_fallback = 1;
+  f.stall_tile = -1;
+  if (tc::mla_pair_supported(c)) {
+    e = tc::launch_decode_mla_pair(map, a, st);
+    if (e != cudaSuccess) return e;
+    f.n_groups = tc::mla_groups(c);
+    return tc::launch_decode_tc_mla(map, f, st);
+  }
+  if (c.d_cb == 512) return tc::launch_decode_tc_mla(map, a, st);
+  if (use_wide(c)) {
+    e = tc::launch_decode_wide(map, a, st);
+    if (e != cudaSuccess || !rows_supported(c)) return e;
+    f.n_groups = (c.n_blocks / g_of(c)) * (c.n_heads / hpc_of(c));
+    return launch_rows(map, f, st);
+  }
+  return launch_rows(map, a, st);
 }
 
 }  // namespace mlra

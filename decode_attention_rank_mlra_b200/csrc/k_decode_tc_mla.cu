@@ -74,7 +74,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
-  int32_t* err = &hdr->error;
+  if (a.range_fallback) {
+    // after the 128-head kernel's grid: every thread reads its final error word
+    pdl_wait();
+    if (*reinterpret_cast<volatile int32_t*>(&hdr->error) != MLRA_ERR_RANGE) return;
+  }
+  int32_t* err = a.range_fallback ? &hdr->fallback_error : &hdr->error;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -446,6 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if (a.range_fallback && threadIdx.x == 0) {
+    // the last CTA out replaces MLRA_ERR_RANGE by this launch's own outcome
+    __threadfence();
+    if (atomicAdd(&hdr->fallback_done, 1) == int(gridDim.x) - 1)
+      atomicCAS(&hdr->error, MLRA_ERR_RANGE,
+                *reinterpret_cast<volatile int32_t*>(&hdr->fallback_error));
   }
 }
 

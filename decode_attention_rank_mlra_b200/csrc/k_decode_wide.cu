@@ -16,7 +16,8 @@
 //    into a multi-stage shared-memory ring;
 //  * warps 8, 10, 11, 13 convert each arrived tile's two latent boxes from bf16 to fp16
 //    in place and zero the rows past the sequence end (exact for
-//    2^-17 <= |c| < 65520; larger magnitudes are reported as MLRA_ERR_RANGE);
+//    2^-17 <= |c| < 65520; larger magnitudes are reported as MLRA_ERR_RANGE, and
+//    the head-rows kernel launched after this one then recomputes the call);
 //  * warp 9 issues tcgen05.mma: S = Q . C^T with the 128 MMA rows = the 128
 //    heads, the queries in TMEM (A) and the tile K-major in shared memory (B):
 //    8 MMAs with the fp16 query against the fp16 latent block (one row per

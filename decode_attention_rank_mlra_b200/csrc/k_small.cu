@@ -55,6 +55,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   // (it does not wait for this kernel and may record an error at once)
   if (threadIdx.x == 0) {
     hdr->error = 0;
+    hdr->fallback_error = 0;
+    hdr->fallback_done = 0;
     __threadfence();
     s_bad = 0;
   }

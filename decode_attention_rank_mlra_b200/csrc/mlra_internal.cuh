@@ -30,7 +30,12 @@ struct WsHeader {
   int32_t ctas_per_group; // persistent CTAs per branch group
   int32_t batch;
   int32_t max_slots;
-  int32_t pad[57];
+  // A launch that recomputes the call on the head-rows (or 64-head MLA) kernel
+  // after a 128-head kernel reported MLRA_ERR_RANGE records its own errors
+  // here, and its CTAs count themselves out here.
+  int32_t fallback_error;
+  int32_t fallback_done;
+  int32_t pad[55];
 };
 static_assert(sizeof(WsHeader) == 256, "header must be 256 bytes");
 
@@ -272,6 +277,10 @@ struct DecodeArgs {
   // MMA warp's bounded wait runs out (MLRA_ERR_TIMEOUT).  -1: none.  Set only
   // from MLRA_TEST_STALL_TILE; honoured by the head-rows kernel.
   int32_t stall_tile = -1;
+  // 1: this launch runs only if the 128-head kernel launched just before it
+  // left MLRA_ERR_RANGE in the error word, and then recomputes every output of
+  // the call (same plan, same slots); otherwise each CTA returns at once.
+  int32_t range_fallback = 0;
 };
 
 }  // namespace mlra

@@ -72,7 +72,13 @@ typedef enum {
   MLRA_ERR_RANGE = 9         /* device: a cache value of magnitude >= 65520 met
                                 a tensor-core kernel that takes the tile as
                                 fp16 (128 heads per CTA; MLA with a multiple
-                                of 128 heads): the result is not usable     */
+                                of 128 heads).  mlra_decode_attn then
+                                recomputes the call with a kernel that keeps
+                                the tile in bf16 (launched right after, it
+                                returns at once unless needed) and the word
+                                reads 0; it stays set, and the result is not
+                                usable, only for MLRA with a multiple of 128
+                                heads above 128, which no bf16 kernel takes */
 } mlra_status_t;
 
 typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype_t;

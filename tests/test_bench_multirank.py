@@ -168,3 +168,24 @@ def test_default_headline_is_the_largest_workload():
     assert bench.split_workloads("all", bench.DEFAULT_WORKLOAD) == [
         n for n in bench.PER_CONFIG if n != bench.DEFAULT_WORKLOAD]
     assert bench.split_workloads("none", bench.DEFAULT_WORKLOAD) == []
+
+
+def test_batch_option_runs_a_smaller_case_of_the_same_workload():
+    """--batch N keeps the workload's shape, layout and length law with N sequences."""
+    import bench
+    import workloads as W
+    a = bench.parse(["--workload", "mlra4_bf16_b128_h16_ragged1k_64k_paged", "--batch", "16"])
+    full, small = W.WORKLOADS[a.workload], bench.workload_spec(W, a)
+    assert small.batch == 16 and small.ragged == full.ragged and small.paged == full.paged
+    assert (small.n_heads, small.n_blocks, small.d_cb, small.d_r) == (
+        full.n_heads, full.n_blocks, full.d_cb, full.d_r)
+    assert bench.workload_spec(W, bench.parse(["--workload", a.workload])) is full
+
+
+def test_launch_count_includes_the_range_recompute_launch_at_128_heads():
+    import bench
+    import workloads as W
+    counts = {n: bench.kernels_per_step(W.WORKLOADS[n]) for n in bench.PER_CONFIG}
+    assert counts["mla_bf16_b8_h128_l131072_paged"] == 5
+    assert counts["mlra4_bf16_b8_h128_l131072_paged"] == 5
+    assert counts["mlra4_bf16_b128_h16_ragged1k_64k_paged"] == 4

@@ -176,10 +176,11 @@ def test_h128_paged_tail_rows_never_matter():
         assert torch.equal(got[k], ref[k]), k
 
 
-def test_h128_cache_values_beyond_fp16_range_are_reported():
-    """The 128-head kernel carries the latent tile into P . C as fp16: a valid
-    cache value of magnitude >= 65520 is reported (MLRA_ERR_RANGE); 59904 is
-    still exact and matches the oracle."""
+def test_h128_cache_values_beyond_fp16_range_are_recomputed():
+    """The 128-head MLRA-4 kernel carries the latent tile into the MMAs as fp16:
+    59904 (bf16) is still exact there; a valid cache value of magnitude >= 65520
+    makes it report MLRA_ERR_RANGE, and the head-rows kernel launched after it
+    recomputes the call in bf16, which then matches the oracle with no error."""
     inp = _small("mlra4_bf16_b8_h128_l131072_paged", 2, [200, 90])
     flat = inp.kv_cache.view(-1, inp.spec.D)
     row = int(inp.page_table[0, 1].item()) * 64 + 3
@@ -188,8 +189,24 @@ def test_h128_cache_values_beyond_fp16_range_are_reported():
     assert got["device_error"] == 0
     compare_batch(inp, got, heads=[0, 1, 64, 127])
     flat[row, 5] = 70000.0          # bf16 70144: outside
-    got = run_gpu(inp)
-    assert got["device_error"] == 9  # MLRA_ERR_RANGE
+    row2 = int(inp.page_table[1, 0].item()) * 64 + 7
+    flat[row2, 300] = -250000.0
+    for fused in (False, True):
+        got = run_gpu(inp, fused=fused)
+        assert got["device_error"] == 0
+        compare_batch(inp, got, heads=[0, 1, 64, 127])
+
+
+def test_mla_h128_cache_values_beyond_fp16_range_are_recomputed():
+    """The same for the paired MLA kernel: a cache value beyond the fp16 range
+    is recomputed by the 64-head MLA kernel (bf16 hi + lo), no error left."""
+    inp = _small("mla_bf16_b8_h128_l131072_paged", 2, [150, 70], seed=7)
+    flat = inp.kv_cache.view(-1, inp.spec.D)
+    flat[int(inp.page_table[0, 1].item()) * 64 + 9, 17] = 70000.0
+    flat[int(inp.page_table[1, 0].item()) * 64 + 2, 400] = -250000.0
+    got = run_gpu(inp, fused=True)
+    assert got["device_error"] == 0
+    compare_batch(inp, got, heads=[0, 63, 64, 127])
 
 
 def test_mla_tile_boundaries():
