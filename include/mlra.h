@@ -180,6 +180,11 @@ MLRA_API mlra_status_t mlra_workspace_size(const mlra_config_t* cfg, int32_t bat
  * reset at the start of every call.  kv_cache, q_abs and q_rope must be
  * 16-byte aligned (they are read in 16-byte units, the cache by the tensor
  * memory accelerator); seqlens and page_table 4-byte aligned.
+ * Launches: the planner and the attention kernel; with bf16 data and 128 heads
+ * (MLRA with d_cb = 128, or MLA with a multiple of 128 heads), whose kernel
+ * takes the tile as fp16, a third launch that returns at once unless a cache
+ * value left the fp16 range (MLRA_ERR_RANGE), in which case it recomputes the
+ * call with a kernel that keeps the tile in bf16 and clears that error.
  */
 MLRA_API mlra_status_t mlra_decode_attn(const mlra_config_t* cfg, const float* q_abs, const void* q_rope,
                                const void* kv_cache, int64_t num_pages, const int32_t* page_table,
