@@ -66,6 +66,17 @@ def test_bf16_h128_oracle_sized(name, fused):
     compare_batch(inp, got, heads=[0, 1, 63, 100, 127])
 
 
+@pytest.mark.parametrize("name", ["mlra4_bf16_b8_h128_l131072_paged", "mla_bf16_b8_h128_l131072_paged"])
+def test_bf16_two_groups_of_128_heads(name):
+    """256 heads: two groups of 128 (two head groups of 128-head CTAs per branch
+    for MLRA-4, two head groups of clusters for MLA), heads on both sides of the
+    group boundary."""
+    inp = _small(name, 2, [700, 129], heads=256, seed=23)
+    got = run_gpu(inp, fused=True)
+    assert got["device_error"] == 0
+    compare_batch(inp, got, heads=[0, 127, 128, 200, 255])
+
+
 @pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("batch", [17, 70, 300])
 def test_batches_spanning_several_sequence_tiles(batch, fused):
