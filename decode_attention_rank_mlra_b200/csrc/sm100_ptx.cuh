@@ -189,21 +189,11 @@ __device__ __forceinline__ void tmem_st_x2_32(uint32_t taddr, const uint32_t (&r
 #undef MLRA_R8
 #undef MLRA_W8
 
-// ---- tcgen05.mma -------------------------------------------------------------
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, one CTA; lanes whose bit is set
-// in the 128-bit mask (m0: lanes 0-31, ... m3: lanes 96-127) are not written.
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate, uint32_t m0,
-                                       uint32_t m1, uint32_t m2, uint32_t m3) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-          d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1), "r"(m2), "r"(m3)
-      : "memory");
-}
-// Same MMA issued by the whole (converged) warp: one elected lane issues it, so
-// the operands stay warp-uniform and the issue path stays short.
+// ---- tcgen05.mma ------------------------------------------------------------
+// D[tmem] (+)= A[tmem] * B[smem desc] (kind::f16, fp32 accumulation), lanes
+// whose mask bit is set skip their output row.  Issued by the whole (converged)
+// warp: one elected lane issues it, so the operands stay warp-uniform and the
+// issue path stays short.
 __device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate, uint32_t m0,
                                             uint32_t m1, uint32_t m2, uint32_t m3) {
@@ -252,12 +242,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Arrive on `bar` once every previously issued tcgen05 op of this thread is done.
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-      : "memory");
-}
 
 // 32-byte store of eight fp32 (full sector; the address is 32-byte aligned).
 __device__ __forceinline__ void st_global_v8(float* p, const float (&v)[8]) {
@@ -283,20 +267,6 @@ __device__ __forceinline__ uint32_t dsmem_addr(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
-}
-// Store 16 / 4 bytes into another CTA's shared memory (addresses from mapa);
-// the bytes count toward the transaction count of that CTA's mbarrier `bar`.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
-                   addr),
-               "r"(v), "r"(bar)
-               : "memory");
 }
 // Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
 // this CTA's shared memory into another CTA's (addresses from mapa); the bytes
@@ -329,16 +299,6 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
-}
-// Commit from the elected lane, arriving on the mbarrier at the same offset in
-// every CTA of `mask` (cluster ranks) once this thread's MMAs are done.
-__device__ __forceinline__ void mma_commit_multicast_warp(uint32_t bar, uint16_t mask) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;\n\t}" ::"r"(bar),
-      "h"(mask)
-      : "memory");
 }
 // 16-byte shared-memory load / store by shared-window address.  (Measured on
 // the converter loop: these explicit forms, two chunks in flight at a time, ran
