@@ -11,10 +11,10 @@
 // absorbed "MQA-style" step of Main Findings ("three absorbable steps").
 //
 // How (one CTA per SM, persistent over a share of the tile stream):
-//  * warp 12 streams 64-token tiles of the cache with TMA (SWIZZLE_128B boxes of
+//  * warp 13 streams 64-token tiles of the cache with TMA (SWIZZLE_128B boxes of
 //    64 rows x 64 columns): the two boxes of latent block c_b and the RoPE box,
 //    into a multi-stage shared-memory ring;
-//  * warps 8, 10, 11, 13 convert each arrived tile's two latent boxes from bf16 to fp16
+//  * warps 8, 10, 11 convert each arrived tile's two latent boxes from bf16 to fp16
 //    in place and zero the rows past the sequence end (exact for
 //    2^-17 <= |c| < 65520; larger magnitudes are reported as MLRA_ERR_RANGE, and
 //    the head-rows kernel launched after this one then recomputes the call);
@@ -45,12 +45,15 @@ using tc::kSmemLimit;
 using tc::wait_bar;
 using tc::wait_bar_warp;
 
-constexpr int kThreadsW = 448;                // warps 0-7 softmax, 8, 10, 11, 13 convert, 9 MMA, 12 TMA
-// One converter warp per scheduler (warp w runs on scheduler w % 4), beside
-// the two softmax warps there: converters 8, 10, 11, 13, MMA warp 9, TMA warp 12.
-constexpr int kWarpTma = 12, kWarpMma = 9;
-__device__ __forceinline__ bool is_conv(int w) { return w == 8 || w == 10 || w == 11 || w == 13; }
-__device__ __forceinline__ int conv_index(int w) { return w == 8 ? 0 : w == 13 ? 3 : w - 9; }
+constexpr int kThreadsW = 448;  // warps 0-7 softmax, 8, 10, 11 convert, 9 MMA, 13 TMA, 12 idle
+// Warp w runs on scheduler w % 4.  The softmax warps of the slowest scheduler
+// gate every tile, so the other roles are spread thin: one converter on
+// schedulers 0, 2 and 3 each, the MMA and TMA warps (light issue) on 1.
+// (Measured: a converter beside the MMA warp, or two on one scheduler, left that
+// scheduler's softmax warps 700-2,000 cycles behind the others.)
+constexpr int kWarpTma = 13, kWarpMma = 9, kConvWarps = 3;
+__device__ __forceinline__ bool is_conv(int w) { return w == 8 || w == 10 || w == 11; }
+__device__ __forceinline__ int conv_index(int w) { return w == 8 ? 0 : w - 9; }
 constexpr uint32_t kTmemColsW = 512;
 constexpr uint32_t kColQ = 0;                 // fp16 query (64 cols) | bf16 RoPE query (32)
 constexpr uint32_t kColQr = 64;
@@ -108,7 +111,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
     for (int i = 0; i < NST; ++i) {
       mbar_init(FULL(i), 1);
       mbar_init(EMPTY(i), 1);
-      mbar_init(CONV(i), 4);
+      mbar_init(CONV(i), kConvWarps);
     }
     for (int i = 0; i < kNS; ++i) {
       mbar_init(SFULL(i), 1);
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
     // The tile's two latent boxes bf16 -> fp16 in place (16-byte chunks in
     // address order); rows past the valid tokens, latent and RoPE, become
     // zeros, so they never depend on what the cache holds there.
-    const int ct = 32 * conv_index(warp) + lane;  // 0..127
+    const int ct = 32 * conv_index(warp) + lane;  // 0..95
     Piece p;
     int it = 0;
     bool ok = true;
@@ -205,8 +208,8 @@ __global__ void __launch_bounds__(kThreadsW, 1)
         if (!wait_bar_warp(FULL(st), (it / NST) & 1, abort_flag, err)) { ok = false; break; }
         const int valid = min(kTile, p.L - t * kTile);
         const uint32_t base = smem_addr(stages + st * STAGE);
-        const uint32_t over = tc::convert_stage<2 * 512, 128>(base, ct, valid);
-        if (valid < kTile) tc::zero_box_rows<128>(base + 2 * kBoxBytes, ct, valid);
+        const uint32_t over = tc::convert_stage<2 * 512, 32 * kConvWarps>(base, ct, valid);
+        if (valid < kTile) tc::zero_box_rows<32 * kConvWarps>(base + 2 * kBoxBytes, ct, valid);
         if ((over & 0x80008000u) != 0) set_error(err, MLRA_ERR_RANGE);
         fence_proxy_async_smem();
         __syncwarp();
@@ -292,7 +295,7 @@ __global__ void __launch_bounds__(kThreadsW, 1)
       while (!mbar_try_wait(DRAIN, 0) && globaltimer() - t0 < 10000000ull) {}
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warps 0-7
     // Warps q and q + 4 share TMEM lane quadrant q: a thread owns one head
     // (lane = row) and one half of each tile's 64 tokens (x = warp / 4); the

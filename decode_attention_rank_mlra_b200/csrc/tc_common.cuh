@@ -70,23 +70,36 @@ __device__ __forceinline__ uint32_t bf16x8_to_f16(uint4& w) {
 }
 
 // Converter step over one stage: the chunks q = ct, ct + kConvThreads, ... <
-// n_chunks of the latent boxes at shared address `base` (64 rows of 128 bytes
+// kChunks of the latent boxes at shared address `base` (64 rows of 128 bytes
 // per box, chunk q in row (q / 8) mod 64), bf16 -> fp16 in place; rows at or
 // past `valid` become zeros.  Two chunks in flight per thread.
 template <int kChunks, int kConvThreads>
 __device__ __forceinline__ uint32_t convert_stage(uint32_t base, int ct, int valid) {
-  static_assert(kChunks % (2 * kConvThreads) == 0, "chunks split evenly in pairs");
   uint32_t over = 0;
   if (valid >= 64) {
+    if constexpr (kChunks % (2 * kConvThreads) == 0) {
 #pragma unroll
-    for (int i = 0; i < kChunks / kConvThreads; i += 2) {
-      const uint32_t a0 = base + 16u * uint32_t(ct + kConvThreads * i);
-      const uint32_t a1 = a0 + 16u * kConvThreads;
-      uint4 w0 = ptx::lds128(a0), w1 = ptx::lds128(a1);
-      over |= bf16x8_to_f16(w0);
-      over |= bf16x8_to_f16(w1);
-      ptx::sts128(a0, w0);
-      ptx::sts128(a1, w1);
+      for (int i = 0; i < kChunks / kConvThreads; i += 2) {
+        const uint32_t a0 = base + 16u * uint32_t(ct + kConvThreads * i);
+        const uint32_t a1 = a0 + 16u * kConvThreads;
+        uint4 w0 = ptx::lds128(a0), w1 = ptx::lds128(a1);
+        over |= bf16x8_to_f16(w0);
+        over |= bf16x8_to_f16(w1);
+        ptx::sts128(a0, w0);
+        ptx::sts128(a1, w1);
+      }
+    } else {  // a share that does not split into pairs: the last pair may be one chunk
+#pragma unroll
+      for (int q = ct; q < kChunks; q += 2 * kConvThreads) {
+        const uint32_t a0 = base + 16u * uint32_t(q);
+        const bool two = q + kConvThreads < kChunks;
+        uint4 w0 = ptx::lds128(a0), w1 = make_uint4(0u, 0u, 0u, 0u);
+        if (two) w1 = ptx::lds128(a0 + 16u * kConvThreads);
+        over |= bf16x8_to_f16(w0);
+        if (two) over |= bf16x8_to_f16(w1);
+        ptx::sts128(a0, w0);
+        if (two) ptx::sts128(a0 + 16u * kConvThreads, w1);
+      }
     }
   } else {
 #pragma unroll 1
